@@ -1,0 +1,256 @@
+"""Pins of the CPU oracle to facts other than itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with
+something the pages or the mathematics fix: a hand-worked example, a library
+routine on a special case, a closed form, an invariant, or brute force.  The
+same functions are run against mutated copies of the oracle (see
+``test_oracle_mutants.py``) to show that a plausible mistake fails at least
+one of them.
+
+Readings pinned here (gist.science summary of arXiv 2606.10722,
+"1. Architectuur" and "3. Hardware Implicaties"): p = B (A x);
+a_j = sigma(p_j) g_j u_j for kept channels, exactly 0 otherwise;
+y = sum_j a_j W_down[:, j]; per 64-channel bank keep the k largest logits,
+equal logits to the lower index.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+from scipy.special import expit
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _layer(rng, d, d_i, r, scale=1.0):
+    x = rng.standard_normal((3, d))
+    A = rng.standard_normal((r, d)) * scale / math.sqrt(d)
+    B = rng.standard_normal((d_i, r)) / math.sqrt(r)
+    Wg = rng.standard_normal((d_i, d)) / math.sqrt(d)
+    Wu = rng.standard_normal((d_i, d)) / math.sqrt(d)
+    Wd = rng.standard_normal((d_i, d)) / math.sqrt(d_i)
+    return x, A, B, Wg, Wu, Wd
+
+
+def _mask_by_stable_sort(p, bank, k):
+    """Reference top-k: numpy's stable argsort of -p per bank, first k."""
+    T, d_i = p.shape
+    out = np.zeros((T, d_i // bank), np.uint64)
+    for t in range(T):
+        for b in range(d_i // bank):
+            seg = p[t, b * bank:(b + 1) * bank]
+            order = np.argsort(-seg, kind="stable")  # NaN sorts last, ties keep index order
+            w = 0
+            for i in order[:k]:
+                w |= 1 << int(i)
+            out[t, b] = w
+    return out
+
+
+# --------------------------------------------------------------------------- top-k
+
+def pin_topk_golden():
+    cases = json.load(open(os.path.join(GOLDEN, "bank_topk_ties.json")))["cases"]
+    for c in cases:
+        if c["logits"] == "ramp64":
+            p = np.arange(64, dtype=np.float64)[None, :]
+        else:
+            p = np.array([[float(v) for v in c["logits"]]], dtype=np.float64)
+        got = oracle.bank_topk(p, c["bank"], c["k"])
+        assert [int(v) for v in got[0]] == c["expected"], (c, got)
+
+
+def pin_topk_popcount():
+    rng = _rng(1)
+    for bank, k in [(64, 16), (64, 1), (64, 63), (64, 64), (32, 5), (8, 3)]:
+        p = rng.standard_normal((5, bank * 7))
+        m = oracle.bank_topk(p, bank, k)
+        for w in m.ravel():
+            w = int(w)
+            assert bin(w).count("1") == k
+            assert w >> bank == 0
+
+
+def pin_topk_stable_sort():
+    rng = _rng(2)
+    for bank, k in [(64, 16), (16, 4), (64, 40)]:
+        p = rng.standard_normal((6, bank * 5))
+        # force ties and signed zeros into every row
+        p = np.round(p * 2) / 2
+        p[:, ::7] = -0.0
+        p[:, 3::11] = 0.0
+        assert (oracle.bank_topk(p, bank, k) == _mask_by_stable_sort(p, bank, k)).all()
+        # fp32 logits widen exactly: the same rule on float32 data
+        p32 = rng.standard_normal((4, bank * 3)).astype(np.float32)
+        assert (oracle.bank_topk(p32, bank, k)
+                == _mask_by_stable_sort(p32.astype(np.float64), bank, k)).all()
+
+
+def pin_topk_brute_force():
+    """Enumerate every k-subset; the kept set maximises the sum and, among
+    maximal sets, has the lexicographically smallest sorted index tuple.
+    Integer logits make the sums exact and create many ties."""
+    rng = _rng(3)
+    for bank in (4, 6, 8):
+        for k in range(1, bank + 1):
+            p = rng.integers(-3, 4, size=(4, bank * 2)).astype(np.float64)
+            m = oracle.bank_topk(p, bank, k)
+            for t in range(p.shape[0]):
+                for b in range(2):
+                    seg = p[t, b * bank:(b + 1) * bank]
+                    best = max(itertools.combinations(range(bank), k),
+                               key=lambda s: (sum(seg[list(s)]), [-i for i in s]))
+                    want = sum(1 << i for i in best)
+                    assert int(m[t, b]) == want, (seg, k, bin(int(m[t, b])), bin(want))
+
+
+# ----------------------------------------------------------------------- predictor
+
+def pin_predict_matmul():
+    """p = B (A x) equals numpy's (B A) x^T: a different association of the
+    same contraction, on non-square shapes so a transposed factor fails."""
+    rng = _rng(4)
+    x, A, B, *_ = _layer(rng, d=48, d_i=80, r=12)
+    p = oracle.predict(x, A, B)
+    ref = ((B @ A) @ x.T).T
+    assert p.shape == (3, 80)
+    assert np.allclose(p, ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_predict_selector():
+    """Closed form: A = [I_r | 0] and one-hot B rows with B[j][j mod r] = 1
+    give p_j = x[j mod r]."""
+    rng = _rng(5)
+    d, r, d_i = 24, 6, 32
+    x = rng.standard_normal((2, d))
+    A = np.zeros((r, d))
+    A[:, :r] = np.eye(r)
+    B = np.zeros((d_i, r))
+    B[np.arange(d_i), np.arange(d_i) % r] = 1.0
+    p = oracle.predict(x, A, B)
+    assert np.array_equal(p, x[:, np.arange(d_i) % r])
+
+
+def pin_predict_integer_exact():
+    """Small integers: double sums are exact, so p equals numpy's int64 matmul."""
+    rng = _rng(6)
+    x = rng.integers(-4, 5, size=(3, 40))
+    A = rng.integers(-4, 5, size=(9, 40))
+    B = rng.integers(-4, 5, size=(24, 9))
+    p = oracle.predict(x.astype(np.float64), A.astype(np.float64), B.astype(np.float64))
+    assert np.array_equal(p, (B @ (A @ x.T)).T.astype(np.float64))
+
+
+# ------------------------------------------------------------------------- sigmoid
+
+def pin_sigmoid():
+    assert oracle.sigmoid(0.0) == 0.5
+    assert abs(oracle.sigmoid(math.log(3.0)) - 0.75) < 1e-15
+    assert abs(oracle.sigmoid(-math.log(3.0)) - 0.25) < 1e-15
+    for z in np.concatenate([np.linspace(-40, 40, 161), [-700.0, 700.0, 1e-9, -1e-9]]):
+        assert abs(oracle.sigmoid(float(z)) - float(expit(z))) <= 1e-15 * max(1.0, expit(z))
+
+
+# --------------------------------------------------------------------------- forward
+
+def pin_forward_golden():
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    arr = {k: np.array(g[k], dtype=np.float64) for k in ("x", "A", "B", "Wg", "Wu", "Wd")}
+    y, p, m = oracle.forward(arr["x"], arr["A"], arr["B"], arr["Wg"], arr["Wu"], arr["Wd"],
+                             g["bank"], g["k"])
+    assert np.array_equal(p, np.array(g["expected_logits"]))
+    assert [int(v) for v in m[0]] == g["expected_mask"]
+    assert np.allclose(y, np.array(g["expected_y"]), rtol=1e-14, atol=0)
+
+
+def _dense_gated_ffn(x, p, Wg, Wu, Wd, keep):
+    """numpy: y = W_down (keep * sigma(p) * (Wg x) * (Wu x)), W_down = Wd^T."""
+    g = x @ Wg.T
+    u = x @ Wu.T
+    a = keep * expit(p) * g * u
+    W_down = Wd.T
+    return (W_down @ a.T).T
+
+
+def pin_forward_k_equals_bank():
+    """k = bank keeps every channel: the predictor-gated dense FFN (the
+    "Predictor-Gated Dense FFN" stage of the recipe)."""
+    rng = _rng(7)
+    x, A, B, Wg, Wu, Wd = _layer(rng, d=40, d_i=128, r=10)
+    y, p, m = oracle.forward(x, A, B, Wg, Wu, Wd, bank=64, k=64)
+    assert all(int(w) == (1 << 64) - 1 for w in m.ravel())
+    ref = _dense_gated_ffn(x, (B @ (A @ x.T)).T, Wg, Wu, Wd, 1.0)
+    assert np.allclose(y, ref, rtol=1e-11, atol=1e-12)
+
+
+def pin_forward_masked_dense():
+    """Skipping channels equals the dense FFN with the intermediate zeroed
+    outside the mask (numpy), and equals the oracle's own dense-then-mask loop."""
+    rng = _rng(8)
+    for bank, k in [(64, 16), (32, 3), (16, 16), (64, 1)]:
+        x, A, B, Wg, Wu, Wd = _layer(rng, d=36, d_i=192, r=8)
+        y, p, m = oracle.forward(x, A, B, Wg, Wu, Wd, bank=bank, k=k)
+        keep = oracle.mask_to_bool(m, bank).astype(np.float64)
+        assert keep.sum(axis=1).tolist() == [k * (192 // bank)] * 3
+        ref = _dense_gated_ffn(x, p, Wg, Wu, Wd, keep)
+        assert np.allclose(y, ref, rtol=1e-11, atol=1e-12)
+        ydm = oracle.dense_then_mask(x, p, m, Wg, Wu, Wd, bank)
+        assert np.allclose(y, ydm, rtol=1e-11, atol=1e-12)
+
+
+def pin_forward_invariants():
+    """Permuting channels inside each bank (rows of B, Wg, Wu, Wd alike)
+    permutes the mask bits and leaves y unchanged; permuting tokens permutes y;
+    y is linear in Wd."""
+    rng = _rng(9)
+    bank, k = 32, 8
+    x, A, B, Wg, Wu, Wd = _layer(rng, d=28, d_i=128, r=7)
+    y, p, m = oracle.forward(x, A, B, Wg, Wu, Wd, bank, k)
+    perm = np.concatenate([b * bank + rng.permutation(bank) for b in range(128 // bank)])
+    y2, p2, m2 = oracle.forward(x, A, B[perm], Wg[perm], Wu[perm], Wd[perm], bank, k)
+    assert np.array_equal(oracle.mask_to_bool(m2, bank), oracle.mask_to_bool(m, bank)[:, perm])
+    assert np.allclose(y2, y, rtol=1e-12, atol=1e-13)
+    tp = np.array([2, 0, 1])
+    y3, _, m3 = oracle.forward(x[tp], A, B, Wg, Wu, Wd, bank, k)
+    assert np.array_equal(m3, m[tp]) and np.array_equal(y3, y[tp])
+    y4, _, _ = oracle.forward(x, A, B, Wg, Wu, 2.0 * Wd, bank, k)
+    assert np.array_equal(y4, 2.0 * y)
+
+
+def pin_forward_bf16_widening():
+    """bf16 inputs are widened exactly: feeding bf16 bit patterns equals
+    feeding their float64 values."""
+    rng = _rng(10)
+    x, A, B, Wg, Wu, Wd = _layer(rng, d=32, d_i=64, r=8)
+
+    def to_bf16_bits(a):
+        f = a.astype(np.float32).view(np.uint32)
+        # round to nearest even on the upper 16 bits
+        f = ((f + 0x7FFF + ((f >> 16) & 1)) >> 16).astype(np.uint16)
+        return f
+
+    def widen(bits):
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    ins = [to_bf16_bits(a) for a in (x, A, B, Wg, Wu, Wd)]
+    y1, p1, m1 = oracle.forward(*ins, bank=64, k=16)
+    y2, p2, m2 = oracle.forward(*[widen(b) for b in ins], bank=64, k=16)
+    assert np.array_equal(p1, p2) and np.array_equal(m1, m2) and np.array_equal(y1, y2)
+
+
+ALL_PINS = [
+    pin_topk_golden, pin_topk_popcount, pin_topk_stable_sort, pin_topk_brute_force,
+    pin_predict_matmul, pin_predict_selector, pin_predict_integer_exact, pin_sigmoid,
+    pin_forward_golden, pin_forward_k_equals_bank, pin_forward_masked_dense,
+    pin_forward_invariants, pin_forward_bf16_widening,
+]
