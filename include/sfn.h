@@ -1,0 +1,194 @@
+/*
+ * sfn.h -- C ABI of libsfn: the forward pass of the predictor-gated bank-wise
+ * top-k sparse SwiGLU FFN on NVIDIA B200 (sm_100a).
+ *
+ * The method: "Continual LLM Upcycling: A Predictor-Gated Bank-Wise Sparsity
+ * Training Recipe for Dense-to-Sparse LLMs" (arXiv 2606.10722).  Passages are
+ * cited by page and section:
+ *   [arch]  gist.science summary, "Methodologie / 1. Architectuur:
+ *           Predictor-Gated Sparse SwiGLU" -- a low-rank predictor
+ *           R^d -> R^448 -> R^{d_i} acts on the token hidden state before the
+ *           FFN; its logits replace the dense SwiGLU gate; d_i = 14336 is cut
+ *           into fixed banks of 64 with a hard top-16 per bank (d_s = 3584);
+ *           in the forward pass inactive channels are exactly zero.
+ *   [hw]    same page, "3. Hardware Implicaties" -- with dedicated kernels
+ *           the gate, up and down projections all skip inactive channels.
+ *   [abs]   the paper's abstract (catalyzex.com / searcharxiv.com author
+ *           pages) -- per token and layer a low-rank predictor gives
+ *           FFN-channel routing logits; a bank-wise top-k keeps 16 channels
+ *           in every 64-channel bank, 4x sparsity.
+ *
+ * Readings of what the pages leave open (fixed here, identical in the CPU
+ * oracle):
+ *   - the predictor is p = B (A x): no bias, no inner activation;
+ *   - each kept channel j computes a_j = sigma(p_j) * (Wg[j].x) * (Wu[j].x)
+ *     (sigma(p) takes the place of the gate's sigma in silu);
+ *     y = sum_{kept j} a_j * W_down[:, j];
+ *   - banks are contiguous channel ranges [b*bank, (b+1)*bank);
+ *   - a bank keeps the k largest logits; equal logits go to the lower
+ *     channel index; +0 equals -0; NaN ranks below every number.
+ *
+ * Layouts (all row-major and contiguous; every pointer is a DEVICE pointer):
+ *   x      [T][d]        hidden states (bf16 or f32)
+ *   A      [r][d]        first predictor factor
+ *   B      [d_i][r]      second predictor factor
+ *   Wg, Wu [d_i][d]      gate / up projection rows
+ *   Wd     [d_i][d]      DOWN PROJECTION STORED CHANNEL-MAJOR: row j of Wd
+ *                        is column j of W_down ([d][d_i]), i.e. Wd = W_down^T,
+ *                        so the 16 kept channels of a bank are 16 contiguous
+ *                        rows of d elements.
+ *   y      [T][d]        output (same element type as x)
+ *   logits [T][d_i]      float32
+ *   mask   [T][d_i/bank] uint64; bit i of word b is channel b*bank + i;
+ *                        bits at and above `bank` are zero.
+ *
+ * Ownership and execution: the caller owns every buffer; the library keeps
+ * no pointer after a call returns.  Every call only enqueues work on
+ * `stream` (cudaStream_t; NULL is the legacy default stream) and returns
+ * without synchronising; results are ready when the stream is.  No call
+ * copies between host and device.  The only allocations are the
+ * stream-ordered scratch of sfn_sparse_ffn_forward (cudaMallocAsync /
+ * cudaFreeAsync on `stream`); the *_ws variants take caller scratch instead.
+ * Calls on different streams may run concurrently if their outputs and
+ * scratch do not overlap.  Results are deterministic: a fixed reduction
+ * order and no floating-point atomics, so a rerun is bit-identical.
+ *
+ * Errors: every argument is checked on the host before anything is
+ * enqueued; on any error status nothing is written.  T == 0 returns SFN_OK
+ * without enqueueing work (pointers are then not inspected).  A launch
+ * failure is reported as SFN_ERR_CUDA; faults during execution surface at
+ * the caller's next synchronisation, as for any CUDA work.  There is no CPU
+ * fallback: without a usable sm_100 device every compute call returns
+ * SFN_ERR_CUDA.
+ */
+#ifndef SFN_H_
+#define SFN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA
+ * include. */
+typedef struct CUstream_st *sfn_stream_t;
+
+typedef enum sfn_status {
+  SFN_OK = 0,
+  SFN_ERR_INVALID_VALUE = 1, /* T < 0; d, d_i or r <= 0; d_i % bank != 0;
+                                not 1 <= k <= bank <= 64; required pointer
+                                NULL; unknown dtype */
+  SFN_ERR_MISALIGNED = 2,    /* a pointer not 16-byte aligned, or d or r not
+                                a multiple of 16 bytes of its element type */
+  SFN_ERR_UNSUPPORTED = 3,   /* a valid shape outside the built kernels'
+                                limits (d > 16384, r > 2048, d_i > 2^24) */
+  SFN_ERR_WORKSPACE = 4,     /* *_ws scratch NULL, misaligned or smaller than
+                                sfn_workspace_bytes() */
+  SFN_ERR_CUDA = 5           /* a CUDA runtime call or launch failed */
+} sfn_status;
+
+typedef enum sfn_dtype {
+  SFN_DTYPE_BF16 = 0, /* x, A, B, Wg, Wu, Wd, y in bf16; fp32 accumulation */
+  SFN_DTYPE_F32 = 1   /* everything in float32 */
+} sfn_dtype;
+
+/* Static, NUL-terminated description of a status code. */
+const char *sfn_status_string(sfn_status s);
+
+/* ABI version of this header (incremented on any signature change). */
+int sfn_abi_version(void);
+
+/* Number of kernels this library has launched in this process (all
+ * devices, all threads).  Diagnostic counter; never reset. */
+uint64_t sfn_kernel_launch_count(void);
+
+/*
+ * Predictor logits [arch]: for every token t, h = A x_t (R^d -> R^r), then
+ * logits[t] = B h (R^r -> R^{d_i}).  Accumulation is float32; h is kept in
+ * float32 between the two factors.
+ * sfn_predict: x, A, B are bf16 (uint16 bit patterns); sfn_predict_f32:
+ * float32.  logits is float32 [T][d_i].
+ */
+sfn_status sfn_predict(const void *x, const void *A, const void *B, float *logits,
+                       int64_t T, int d, int d_i, int r, sfn_stream_t stream);
+sfn_status sfn_predict_f32(const float *x, const float *A, const float *B, float *logits,
+                           int64_t T, int d, int d_i, int r, sfn_stream_t stream);
+
+/*
+ * Bank-wise hard top-k [arch], [abs]: in every bank of `bank` consecutive
+ * channels of logits[t], set the bits of the k largest logits (ties to the
+ * lower index, NaN lowest).  Exactly k bits are set in every word.
+ * logits float32 [T][d_i] -> mask uint64 [T][d_i/bank].
+ */
+sfn_status sfn_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,
+                         int bank, int k, sfn_stream_t stream);
+
+/*
+ * Bytes of scratch the *_ws forward variants need for this shape and
+ * element type (0 when T == 0).  Returns 0 for invalid arguments.
+ */
+size_t sfn_workspace_bytes(int64_t T, int d, int d_i, int r, int bank, int k,
+                           sfn_dtype dtype);
+
+/*
+ * The whole sparse FFN forward [arch], [hw]: predictor logits, bank-wise
+ * top-k mask, then for the kept channels only a_j = sigma(p_j) * (Wg[j].x) *
+ * (Wu[j].x) and y = sum_j a_j Wd[j, :].  Unkept channels are never read.
+ * x, A, B, Wg, Wu, Wd, y are bf16 (uint16 bit patterns); mask, if not NULL,
+ * receives the mask used.  Scratch is taken stream-ordered from the
+ * device's default memory pool and returned before the call's work ends.
+ */
+sfn_status sfn_sparse_ffn_forward(const void *x, const void *A, const void *B,
+                                  const void *Wg, const void *Wu, const void *Wd, void *y,
+                                  uint64_t *mask, int64_t T, int d, int d_i, int r,
+                                  int bank, int k, sfn_stream_t stream);
+
+/* As sfn_sparse_ffn_forward, with caller scratch `workspace` (device, 256-byte
+ * aligned, at least sfn_workspace_bytes(..., SFN_DTYPE_BF16) bytes).  The
+ * scratch must not be used by other work until this call's work is done. */
+sfn_status sfn_sparse_ffn_forward_ws(const void *x, const void *A, const void *B,
+                                     const void *Wg, const void *Wu, const void *Wd,
+                                     void *y, uint64_t *mask, int64_t T, int d, int d_i,
+                                     int r, int bank, int k, void *workspace,
+                                     size_t workspace_bytes, sfn_stream_t stream);
+
+/* float32 twins of the two forward entry points. */
+sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
+                                      const float *Wg, const float *Wu, const float *Wd,
+                                      float *y, uint64_t *mask, int64_t T, int d, int d_i,
+                                      int r, int bank, int k, sfn_stream_t stream);
+sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const float *B,
+                                         const float *Wg, const float *Wu, const float *Wd,
+                                         float *y, uint64_t *mask, int64_t T, int d,
+                                         int d_i, int r, int bank, int k, void *workspace,
+                                         size_t workspace_bytes, sfn_stream_t stream);
+
+/*
+ * Per-stage timing (diagnostics; no counterpart in the paper).  Between
+ * sfn_timing_begin() and sfn_timing_end(), every kernel the library launches
+ * is bracketed by two CUDA events recorded on its stream.  sfn_timing_end()
+ * waits for those events, then writes for each stage s < n the summed
+ * kernel time in milliseconds (ms[s]) and the number of launches
+ * (launches[s]); either array may be NULL.  Not for use during stream
+ * capture.  Process-wide; not meant for concurrent use from several threads.
+ * Stage ids are the SFN_STAGE_* values; sfn_stage_name() names them.
+ */
+enum {
+  SFN_STAGE_PRED_H = 0,       /* h = A x                                */
+  SFN_STAGE_LOGITS_TOPK = 1,  /* p = B h, bank top-k, sigma(p) of kept  */
+  SFN_STAGE_GATHER_FFN = 2,   /* kept gate/up rows, a_j, kept down rows */
+  SFN_STAGE_REDUCE = 3,       /* sum of partial output rows -> y        */
+  SFN_STAGE_BANK_TOPK = 4,    /* standalone top-k on given logits       */
+  SFN_STAGE_COUNT = 16        /* room for the stage ids of this library */
+};
+sfn_status sfn_timing_begin(void);
+sfn_status sfn_timing_end(double *ms, uint64_t *launches, int n);
+const char *sfn_stage_name(int stage);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFN_H_ */

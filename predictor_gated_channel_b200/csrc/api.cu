@@ -1,0 +1,395 @@
+// api.cu -- the extern "C" entry points of libsfn: argument validation,
+// scratch layout and kernel dispatch.  Every check happens before anything
+// is enqueued, so an error status means nothing was written.
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "sfn_internal.cuh"
+
+namespace sfn {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_dev_mu;
+DeviceInfo g_dev_cache[64];
+
+// CTAs the gather kernel aims for (two per SM of a 148-SM part); fixed so
+// that the scratch size does not depend on the device.
+constexpr int kGatherTargetCtas = 296;
+// Shape limits of the built kernels (shared-memory staging of x, h).
+constexpr int kMaxD = 16384;
+constexpr int kMaxR = 2048;
+constexpr int kMaxDi = 1 << 24;
+constexpr size_t kStageBudget = 96 * 1024;  // bytes of x rows staged per CTA
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// ---- optional per-stage timing (sfn_timing_begin / sfn_timing_end)
+struct TimingRec {
+  int stage;
+  cudaEvent_t start, stop;
+};
+std::mutex g_tmu;
+std::atomic<bool> g_timing{false};
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Run one launcher; when timing is on, bracket it with events on `st`.
+template <class F>
+cudaError_t timed(int stage, cudaStream_t st, F &&launch) {
+  if (!g_timing.load(std::memory_order_relaxed)) return launch();
+  std::lock_guard<std::mutex> lock(g_tmu);
+  cudaEvent_t a = take_event(), b = take_event();
+  if (a) cudaEventRecord(a, st);
+  cudaError_t e = launch();
+  if (b) cudaEventRecord(b, st);
+  if (a && b) g_recs.push_back({stage, a, b});
+  return e;
+}
+
+int pow2_tokens(int64_t T, int cap) {
+  int tt = 1;
+  while (tt < cap && tt < T) tt *= 2;
+  return tt;
+}
+}  // namespace
+
+void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+cudaError_t ensure_smem_limit(const void *kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  struct Key {
+    const void *k;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Key> done;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Key &kk : done)
+    if (kk.k == kernel && kk.dev == dev && kk.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.push_back({kernel, dev, bytes});
+  return e;
+}
+
+bool device_info(DeviceInfo *out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo &c = g_dev_cache[dev];
+  if (c.device != dev) {
+    int major = 0, sms = 0, smem = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return false;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return false;
+    if (cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+      return false;
+    if (major != 10) return false;  // the library is built for sm_100a only
+    c.num_sms = sms;
+    c.max_smem_optin = smem;
+    c.device = dev;
+  }
+  *out = c;
+  return true;
+}
+
+GatherPlan plan_gather(const FwdShape &s) {
+  GatherPlan p{};
+  int tt = pow2_tokens(s.T, 8);
+  while (tt > 1 && (size_t)tt * s.d * sizeof(float) > kStageBudget) tt /= 2;
+  p.tt_h = tt;
+  p.tt_p = pow2_tokens(s.T, 8);
+  int64_t nc = (kGatherTargetCtas + s.T - 1) / s.T;
+  nc = std::min<int64_t>(nc, (s.d_s + 3) / 4);
+  nc = std::max<int64_t>(nc, 1);
+  p.chunk = (int)((s.d_s + nc - 1) / nc);
+  p.n_chunks = (s.d_s + p.chunk - 1) / p.chunk;
+  size_t off = 0;
+  p.off_h = off;
+  off = align_up(off + (size_t)s.T * s.r * sizeof(float), 256);
+  p.off_idx = off;
+  off = align_up(off + (size_t)s.T * s.d_s * sizeof(int), 256);
+  p.off_sig = off;
+  off = align_up(off + (size_t)s.T * s.d_s * sizeof(float), 256);
+  p.off_part = off;
+  off = align_up(off + (size_t)s.T * p.n_chunks * s.d * sizeof(float), 256);
+  p.off_mask = off;
+  p.total = off;
+  return p;
+}
+
+}  // namespace sfn
+
+using namespace sfn;
+
+namespace {
+
+sfn_status check_shape(int64_t T, int d, int d_i, int r, int bank, int k) {
+  if (T < 0 || d <= 0 || d_i <= 0 || r <= 0) return SFN_ERR_INVALID_VALUE;
+  if (bank < 1 || bank > 64 || k < 1 || k > bank || d_i % bank != 0)
+    return SFN_ERR_INVALID_VALUE;
+  return SFN_OK;
+}
+
+sfn_status check_limits(int d, int d_i, int r) {
+  if (d > kMaxD || r > kMaxR || d_i > kMaxDi) return SFN_ERR_UNSUPPORTED;
+  return SFN_OK;
+}
+
+sfn_status check_rows(int d, int r, bool bf16) {
+  const int elt = bf16 ? 2 : 4;
+  if ((d * elt) % 16 != 0 || (r * elt) % 16 != 0) return SFN_ERR_MISALIGNED;
+  return SFN_OK;
+}
+
+FwdShape make_shape(int64_t T, int d, int d_i, int r, int bank, int k, bool bf16) {
+  FwdShape s;
+  s.T = T;
+  s.d = d;
+  s.d_i = d_i;
+  s.r = r;
+  s.bank = bank;
+  s.k = k;
+  s.n_banks = d_i / bank;
+  s.d_s = s.n_banks * k;
+  s.bf16 = bf16;
+  return s;
+}
+
+sfn_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SFN_OK;
+  cudaGetLastError();  // clear a sticky launch error of our own making
+  return SFN_ERR_CUDA;
+}
+
+sfn_status predict_impl(const void *x, const void *A, const void *B, float *logits, int64_t T,
+                        int d, int d_i, int r, bool bf16, cudaStream_t st) {
+  sfn_status s0 = check_shape(T, d, d_i, r, 1, 1);
+  if (s0 != SFN_OK) return s0;
+  if ((s0 = check_limits(d, d_i, r)) != SFN_OK) return s0;
+  if ((s0 = check_rows(d, r, bf16)) != SFN_OK) return s0;
+  if (T == 0) return SFN_OK;
+  if (!x || !A || !B || !logits) return SFN_ERR_INVALID_VALUE;
+  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(logits, 4))
+    return SFN_ERR_MISALIGNED;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return SFN_ERR_CUDA;
+  FwdShape s = make_shape(T, d, d_i, r, 1, 1, bf16);
+  GatherPlan p = plan_gather(s);
+  float *h = nullptr;
+  if (cudaMallocAsync((void **)&h, (size_t)T * r * sizeof(float), st) != cudaSuccess)
+    return cuda_status(cudaErrorMemoryAllocation);
+  cudaError_t e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
+      return launch_logits_topk(s, p.tt_p, h, B, logits, nullptr, nullptr, nullptr, st);
+    });
+  cudaError_t ef = cudaFreeAsync(h, st);
+  if (e == cudaSuccess) e = ef;
+  return cuda_status(e);
+}
+
+sfn_status forward_impl(const void *x, const void *A, const void *B, const void *Wg,
+                        const void *Wu, const void *Wd, void *y, uint64_t *mask, int64_t T,
+                        int d, int d_i, int r, int bank, int k, bool bf16, void *ws,
+                        size_t ws_bytes, bool own_ws, cudaStream_t st) {
+  sfn_status s0 = check_shape(T, d, d_i, r, bank, k);
+  if (s0 != SFN_OK) return s0;
+  if ((s0 = check_limits(d, d_i, r)) != SFN_OK) return s0;
+  if ((s0 = check_rows(d, r, bf16)) != SFN_OK) return s0;
+  if (T == 0) return SFN_OK;
+  if (!x || !A || !B || !Wg || !Wu || !Wd || !y) return SFN_ERR_INVALID_VALUE;
+  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(Wg, 16) ||
+      !aligned(Wu, 16) || !aligned(Wd, 16) || !aligned(y, 16) ||
+      (mask && !aligned(mask, 8)))
+    return SFN_ERR_MISALIGNED;
+  FwdShape s = make_shape(T, d, d_i, r, bank, k, bf16);
+  GatherPlan p = plan_gather(s);
+  if (!own_ws && (ws == nullptr || !aligned(ws, 256) || ws_bytes < p.total))
+    return SFN_ERR_WORKSPACE;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return SFN_ERR_CUDA;
+  if (own_ws && cudaMallocAsync(&ws, p.total, st) != cudaSuccess)
+    return cuda_status(cudaErrorMemoryAllocation);
+  char *w = static_cast<char *>(ws);
+  float *h = reinterpret_cast<float *>(w + p.off_h);
+  int *sel_idx = reinterpret_cast<int *>(w + p.off_idx);
+  float *sel_sig = reinterpret_cast<float *>(w + p.off_sig);
+  float *partial = reinterpret_cast<float *>(w + p.off_part);
+
+  cudaError_t e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
+      return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, st);
+    });
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_GATHER_FFN, st, [&] {
+      return launch_gather_ffn(s, p, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, st);
+    });
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_REDUCE, st, [&] { return launch_reduce(s, p, partial, y, st); });
+  if (own_ws) {
+    cudaError_t ef = cudaFreeAsync(ws, st);
+    if (e == cudaSuccess) e = ef;
+  }
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sfn_status_string(sfn_status s) {
+  switch (s) {
+    case SFN_OK: return "SFN_OK: success";
+    case SFN_ERR_INVALID_VALUE: return "SFN_ERR_INVALID_VALUE: invalid shape, k, bank or pointer";
+    case SFN_ERR_MISALIGNED: return "SFN_ERR_MISALIGNED: pointer or row not 16-byte aligned";
+    case SFN_ERR_UNSUPPORTED: return "SFN_ERR_UNSUPPORTED: shape outside the built kernels' limits";
+    case SFN_ERR_WORKSPACE: return "SFN_ERR_WORKSPACE: scratch missing, misaligned or too small";
+    case SFN_ERR_CUDA: return "SFN_ERR_CUDA: CUDA call or launch failed";
+  }
+  return "unknown sfn_status";
+}
+
+int sfn_abi_version(void) { return 1; }
+
+uint64_t sfn_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+sfn_status sfn_predict(const void *x, const void *A, const void *B, float *logits, int64_t T,
+                       int d, int d_i, int r, sfn_stream_t stream) {
+  return predict_impl(x, A, B, logits, T, d, d_i, r, true, (cudaStream_t)stream);
+}
+
+sfn_status sfn_predict_f32(const float *x, const float *A, const float *B, float *logits,
+                           int64_t T, int d, int d_i, int r, sfn_stream_t stream) {
+  return predict_impl(x, A, B, logits, T, d, d_i, r, false, (cudaStream_t)stream);
+}
+
+sfn_status sfn_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i, int bank,
+                         int k, sfn_stream_t stream) {
+  if (T < 0 || d_i <= 0 || bank < 1 || bank > 64 || k < 1 || k > bank || d_i % bank != 0)
+    return SFN_ERR_INVALID_VALUE;
+  if (d_i > kMaxDi) return SFN_ERR_UNSUPPORTED;
+  if (T == 0) return SFN_OK;
+  if (!logits || !mask) return SFN_ERR_INVALID_VALUE;
+  if (!aligned(logits, 4) || !aligned(mask, 8)) return SFN_ERR_MISALIGNED;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return SFN_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  return cuda_status(timed(SFN_STAGE_BANK_TOPK, st, [&] {
+    return launch_bank_topk(logits, mask, T, d_i, bank, k, st);
+  }));
+}
+
+size_t sfn_workspace_bytes(int64_t T, int d, int d_i, int r, int bank, int k,
+                           sfn_dtype dtype) {
+  if (dtype != SFN_DTYPE_BF16 && dtype != SFN_DTYPE_F32) return 0;
+  if (check_shape(T, d, d_i, r, bank, k) != SFN_OK || T == 0) return 0;
+  if (check_limits(d, d_i, r) != SFN_OK) return 0;
+  return plan_gather(make_shape(T, d, d_i, r, bank, k, dtype == SFN_DTYPE_BF16)).total;
+}
+
+sfn_status sfn_sparse_ffn_forward(const void *x, const void *A, const void *B, const void *Wg,
+                                  const void *Wu, const void *Wd, void *y, uint64_t *mask,
+                                  int64_t T, int d, int d_i, int r, int bank, int k,
+                                  sfn_stream_t stream) {
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, nullptr, 0,
+                      true, (cudaStream_t)stream);
+}
+
+sfn_status sfn_sparse_ffn_forward_ws(const void *x, const void *A, const void *B,
+                                     const void *Wg, const void *Wu, const void *Wd, void *y,
+                                     uint64_t *mask, int64_t T, int d, int d_i, int r,
+                                     int bank, int k, void *workspace, size_t workspace_bytes,
+                                     sfn_stream_t stream) {
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, workspace,
+                      workspace_bytes, false, (cudaStream_t)stream);
+}
+
+sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
+                                      const float *Wg, const float *Wu, const float *Wd,
+                                      float *y, uint64_t *mask, int64_t T, int d, int d_i,
+                                      int r, int bank, int k, sfn_stream_t stream) {
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, false, nullptr, 0,
+                      true, (cudaStream_t)stream);
+}
+
+sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const float *B,
+                                         const float *Wg, const float *Wu, const float *Wd,
+                                         float *y, uint64_t *mask, int64_t T, int d, int d_i,
+                                         int r, int bank, int k, void *workspace,
+                                         size_t workspace_bytes, sfn_stream_t stream) {
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, false, workspace,
+                      workspace_bytes, false, (cudaStream_t)stream);
+}
+
+sfn_status sfn_timing_begin(void) {
+  std::lock_guard<std::mutex> lock(g_tmu);
+  for (auto &r : g_recs) {
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_recs.clear();
+  g_timing.store(true);
+  return SFN_OK;
+}
+
+sfn_status sfn_timing_end(double *ms, uint64_t *launches, int n) {
+  std::lock_guard<std::mutex> lock(g_tmu);
+  g_timing.store(false);
+  if (ms)
+    for (int i = 0; i < n; ++i) ms[i] = 0.0;
+  if (launches)
+    for (int i = 0; i < n; ++i) launches[i] = 0;
+  sfn_status st = SFN_OK;
+  for (auto &r : g_recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) {
+      st = SFN_ERR_CUDA;
+      continue;
+    }
+    if (r.stage >= 0 && r.stage < n) {
+      if (ms) ms[r.stage] += t;
+      if (launches) launches[r.stage] += 1;
+    }
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_recs.clear();
+  if (st != SFN_OK) cudaGetLastError();
+  return st;
+}
+
+const char *sfn_stage_name(int stage) {
+  switch (stage) {
+    case SFN_STAGE_PRED_H: return "pred_h";
+    case SFN_STAGE_LOGITS_TOPK: return "logits_topk";
+    case SFN_STAGE_GATHER_FFN: return "gather_ffn";
+    case SFN_STAGE_REDUCE: return "reduce";
+    case SFN_STAGE_BANK_TOPK: return "bank_topk";
+  }
+  return "unused";
+}
+
+}  // extern "C"

@@ -1,0 +1,273 @@
+// predict_topk.cu -- CUDA-core kernels of the predictor and the bank top-k.
+//
+// Predictor "R^d -> R^448 -> R^{d_i}" and the bank-wise hard top-16 of 64:
+// "Continual LLM Upcycling: A Predictor-Gated Bank-Wise Sparsity Training
+// Recipe for Dense-to-Sparse LLMs", gist.science summary, "1. Architectuur".
+//
+//   k_pred_h       h[t] = A x[t]                (fp32 out, one warp per row of A)
+//   k_logits_topk  p[t] = B h[t] for one bank, then (optionally) that bank's
+//                  top-k: mask word, kept channel ids and sigma(p) in
+//                  ascending channel order (one CTA per bank and token group)
+//   k_bank_topk    standalone top-k on float32 logits (one warp per bank)
+//
+// Every weight element is read with 16-byte loads; accumulation is fp32 in a
+// fixed order.
+#include "sfn_internal.cuh"
+
+namespace sfn {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// Stage TT token rows of x (element type E) into shared memory as float;
+// rows past the end of the batch are zero.
+template <class E, int TT>
+__device__ __forceinline__ void stage_rows(float *xs, const char *x, int64_t t0, int nt,
+                                           int d) {
+  const int nchunk = d / E::kVec;
+  for (int i = threadIdx.x; i < TT * nchunk; i += blockDim.x) {
+    const int t = i / nchunk, c = i - t * nchunk;
+    float f[E::kVec];
+    if (t < nt) {
+      const uint4 v = ld_nc16(x + ((t0 + t) * (int64_t)d + (int64_t)c * E::kVec) * E::kBytes);
+      E::unpack(v, f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E::kVec; ++e) f[e] = 0.f;
+    }
+    float4 *dst = reinterpret_cast<float4 *>(xs + t * d + c * E::kVec);
+#pragma unroll
+    for (int e = 0; e < E::kVec / 4; ++e)
+      dst[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+  }
+}
+
+// h[t][m] = sum_n A[m][n] x[t][n].  1-D grid over (token group, row block):
+// blockIdx.x = token_group * ceil(r / kWarps) + row_block.
+template <class E, int TT>
+__global__ void __launch_bounds__(kThreads) k_pred_h(const char *__restrict__ x,
+                                                     const char *__restrict__ A,
+                                                     float *__restrict__ h, int64_t T, int d,
+                                                     int r) {
+  extern __shared__ float4 smem_f4[];
+  float *xs = reinterpret_cast<float *>(smem_f4);
+  const int row_blocks = (r + kWarps - 1) / kWarps;
+  const int64_t t0 = (int64_t)(blockIdx.x / row_blocks) * TT;
+  const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
+  stage_rows<E, TT>(xs, x, t0, nt, d);
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = (blockIdx.x % row_blocks) * kWarps + warp;
+  if (m >= r) return;
+  const int nchunk = d / E::kVec;
+  const char *row = A + (int64_t)m * d * E::kBytes;
+  float acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+#pragma unroll 4
+  for (int c = lane; c < nchunk; c += 32) {
+    float a[E::kVec];
+    E::unpack(ld_stream16(row + (int64_t)c * 16), a);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      const float *xr = xs + t * d + c * E::kVec;
+#pragma unroll
+      for (int e = 0; e < E::kVec; ++e) acc[t] = fmaf(a[e], xr[e], acc[t]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    const float v = warp_sum(acc[t]);
+    if (lane == 0 && t < nt) h[(t0 + t) * r + m] = v;
+  }
+}
+
+// Logits of one bank for TT tokens, then the bank's top-k.  1-D grid:
+// blockIdx.x = token_group * n_banks + bank_index.
+//   logits  : if kWriteLogits, [T][d_i] float32
+//   mask    : if non-null, [T][n_banks] uint64
+//   sel_idx : if kTopk, [T][d_s] channel ids of kept channels, bank-major,
+//             ascending inside each bank; sel_sig the matching sigma(p)
+template <class E, int TT, bool kWriteLogits, bool kTopk>
+__global__ void __launch_bounds__(kThreads) k_logits_topk(
+    const float *__restrict__ h, const char *__restrict__ B, float *__restrict__ logits,
+    uint64_t *__restrict__ mask, int *__restrict__ sel_idx, float *__restrict__ sel_sig,
+    int64_t T, int d_i, int r, int bank, int k) {
+  extern __shared__ float4 smem_f4[];
+  float *hs = reinterpret_cast<float *>(smem_f4);  // [TT][r]
+  float *ps = hs + TT * r;                         // [TT][64]
+  const int n_banks = d_i / bank;
+  const int b = blockIdx.x % n_banks;
+  const int64_t t0 = (int64_t)(blockIdx.x / n_banks) * TT;
+  const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
+  for (int i = threadIdx.x; i < TT * r; i += blockDim.x) {
+    const int t = i / r;
+    hs[i] = (t < nt) ? h[(t0 + t) * r + (i - t * r)] : 0.f;
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nchunk = r / E::kVec;
+  for (int jl = warp; jl < bank; jl += kWarps) {
+    const int j = b * bank + jl;
+    const char *row = B + (int64_t)j * r * E::kBytes;
+    float acc[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+    for (int c = lane; c < nchunk; c += 32) {
+      float w[E::kVec];
+      E::unpack(ld_stream16(row + (int64_t)c * 16), w);
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const float *hr = hs + t * r + c * E::kVec;
+#pragma unroll
+        for (int e = 0; e < E::kVec; ++e) acc[t] = fmaf(w[e], hr[e], acc[t]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      const float v = warp_sum(acc[t]);
+      if (lane == 0) {
+        ps[t * 64 + jl] = v;
+        if (kWriteLogits && t < nt) logits[(t0 + t) * d_i + j] = v;
+      }
+    }
+  }
+  if (!kTopk) return;
+  __syncthreads();
+
+  const int d_s = n_banks * k;
+  for (int t = warp; t < nt; t += kWarps) {
+    const float p0 = (lane < bank) ? ps[t * 64 + lane] : 0.f;
+    const float p1 = (lane + 32 < bank) ? ps[t * 64 + lane + 32] : 0.f;
+    const uint64_t word = warp_bank_topk(order_key(p0), order_key(p1), bank, k);
+    const int64_t tg = t0 + t;
+    if (mask != nullptr && lane == 0) mask[tg * n_banks + b] = word;
+    int *idx_row = sel_idx + tg * d_s + b * k;
+    float *sig_row = sel_sig + tg * d_s + b * k;
+    if ((word >> lane) & 1ull) {
+      const int s = __popcll(word & ((1ull << lane) - 1ull));
+      idx_row[s] = b * bank + lane;
+      sig_row[s] = sigmoid_f32(p0);
+    }
+    if (lane + 32 < 64 && ((word >> (lane + 32)) & 1ull)) {
+      const int s = __popcll(word & ((1ull << (lane + 32)) - 1ull));
+      idx_row[s] = b * bank + lane + 32;
+      sig_row[s] = sigmoid_f32(p1);
+    }
+  }
+}
+
+// Standalone top-k: one warp per (token, bank).
+__global__ void __launch_bounds__(kThreads) k_bank_topk(const float *__restrict__ logits,
+                                                        uint64_t *__restrict__ mask,
+                                                        int64_t n_words, int bank, int k) {
+  const int64_t wi = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (wi >= n_words) return;  // whole warp leaves together
+  const int lane = threadIdx.x & 31;
+  const float *p = logits + wi * bank;  // banks of a row are contiguous
+  const uint32_t k0 = (lane < bank) ? order_key(p[lane]) : 0u;
+  const uint32_t k1 = (lane + 32 < bank) ? order_key(p[lane + 32]) : 0u;
+  const uint64_t word = warp_bank_topk(k0, k1, bank, k);
+  if (lane == 0) mask[wi] = word;
+}
+
+template <class K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return ensure_smem_limit(reinterpret_cast<const void *>(kernel), bytes);
+}
+
+template <class E, int TT>
+cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, float *h,
+                      cudaStream_t st) {
+  const size_t smem = (size_t)TT * s.d * sizeof(float);
+  auto kern = k_pred_h<E, TT>;
+  cudaError_t e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (int64_t)((s.r + kWarps - 1) / kWarps) * ((s.T + TT - 1) / TT);
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<(unsigned)blocks, kThreads, smem, st>>>((const char *)x, (const char *)A, h, s.T, s.d, s.r);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <class E, int TT, bool W, bool K>
+cudaError_t logits_tt(const FwdShape &s, const float *h, const void *B, float *logits,
+                      uint64_t *mask, int *sel_idx, float *sel_sig, cudaStream_t st) {
+  const size_t smem = (size_t)TT * (s.r + 64) * sizeof(float);
+  auto kern = k_logits_topk<E, TT, W, K>;
+  cudaError_t e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (int64_t)s.n_banks * ((s.T + TT - 1) / TT);
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<(unsigned)blocks, kThreads, smem, st>>>(h, (const char *)B, logits, mask, sel_idx, sel_sig, s.T,
+                                     s.d_i, s.r, s.bank, s.k);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <class E, bool W, bool K>
+cudaError_t logits_dispatch(const FwdShape &s, int tt, const float *h, const void *B,
+                            float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
+                            cudaStream_t st) {
+  switch (tt) {
+    case 1: return logits_tt<E, 1, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
+    case 2: return logits_tt<E, 2, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
+    case 4: return logits_tt<E, 4, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
+    default: return logits_tt<E, 8, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
+                          cudaStream_t st) {
+  if (s.bf16) {
+    switch (tt) {
+      case 1: return pred_h_tt<EltBF16, 1>(s, x, A, h, st);
+      case 2: return pred_h_tt<EltBF16, 2>(s, x, A, h, st);
+      case 4: return pred_h_tt<EltBF16, 4>(s, x, A, h, st);
+      default: return pred_h_tt<EltBF16, 8>(s, x, A, h, st);
+    }
+  }
+  switch (tt) {
+    case 1: return pred_h_tt<EltF32, 1>(s, x, A, h, st);
+    case 2: return pred_h_tt<EltF32, 2>(s, x, A, h, st);
+    case 4: return pred_h_tt<EltF32, 4>(s, x, A, h, st);
+    default: return pred_h_tt<EltF32, 8>(s, x, A, h, st);
+  }
+}
+
+cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,
+                               float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
+                               cudaStream_t st) {
+  const bool topk = sel_idx != nullptr;
+  const bool write = logits != nullptr;
+  if (s.bf16) {
+    if (topk && write)
+      return logits_dispatch<EltBF16, true, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+    if (topk)
+      return logits_dispatch<EltBF16, false, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+    return logits_dispatch<EltBF16, true, false>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+  }
+  if (topk && write)
+    return logits_dispatch<EltF32, true, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+  if (topk)
+    return logits_dispatch<EltF32, false, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+  return logits_dispatch<EltF32, true, false>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+}
+
+cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,
+                             int bank, int k, cudaStream_t st) {
+  const int64_t n_words = T * (d_i / bank);
+  const int64_t blocks = (n_words + kWarps - 1) / kWarps;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  k_bank_topk<<<(unsigned)blocks, kThreads, 0, st>>>(logits, mask, n_words, bank, k);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace sfn

@@ -1,0 +1,161 @@
+// sfn_internal.cuh -- device helpers and host launcher declarations shared by
+// the libsfn translation units.  Nothing here is part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sfn.h"
+
+namespace sfn {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------- elements
+// A 16-byte chunk holds kVec elements; both types unpack to float.
+struct EltBF16 {
+  static constexpr int kVec = 8;
+  static constexpr int kBytes = 2;
+  __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8]) {
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xffff0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xffff0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xffff0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xffff0000u);
+  }
+};
+struct EltF32 {
+  static constexpr int kVec = 4;
+  static constexpr int kBytes = 4;
+  __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[4]) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+};
+
+// float -> bf16 bits, round to nearest even (finite inputs; NaN stays NaN).
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u);
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// Read-only 16-byte load of streamed weights: no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_nc16(const void *p) {
+  return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// Logistic function with CUDA's expf (full-precision library call).
+__device__ __forceinline__ float sigmoid_f32(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+// Order-preserving key of a float logit for the bank ranking: a larger logit
+// gets a larger key, +0 and -0 share one key, every NaN maps to 0, below the
+// key of -inf.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN
+  if ((b << 1) == 0u) b = 0u;                      // -0 -> +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Hard top-k of one bank (bank <= 64) held by a warp: lane l holds the keys
+// of channels l (key0) and l + 32 (key1).  Channel i ranks below channel j
+// when key_j > key_i, or key_j == key_i and j < i; a channel is kept when
+// fewer than k channels rank above it.  Returns the 64-bit keep mask (bit i =
+// channel i), identical in every lane.
+__device__ __forceinline__ uint64_t warp_bank_topk(uint32_t key0, uint32_t key1, int bank,
+                                                   int k) {
+  const int lane = threadIdx.x & 31;
+  int r0 = 0, r1 = 0;
+#pragma unroll 8
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t a = __shfl_sync(kFull, key0, j);  // channel j
+    const uint32_t c = __shfl_sync(kFull, key1, j);  // channel j + 32
+    if (j < bank) {
+      r0 += (a > key0) | ((a == key0) & (j < lane));
+      r1 += (a >= key1);  // channel j < lane + 32 always: ties go to j
+    }
+    if (j + 32 < bank) {
+      r0 += (c > key0);  // channel j + 32 > lane: ties stay with lane
+      r1 += (c > key1) | ((c == key1) & (j < lane));
+    }
+  }
+  const bool s0 = (lane < bank) && (r0 < k);
+  const bool s1 = (lane + 32 < bank) && (r1 < k);
+  const uint32_t lo = __ballot_sync(kFull, s0);
+  const uint32_t hi = __ballot_sync(kFull, s1);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// --------------------------------------------------------------- host side
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  int max_smem_optin = 0;
+};
+// Cached per-device properties; returns false if no device is usable.
+bool device_info(DeviceInfo *out);
+
+void count_launches(uint64_t n);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device, once per (kernel, device, size class); no-op up to 48 KB.
+// Done before the first launch so that no attribute call happens later, for
+// example inside a stream capture.
+cudaError_t ensure_smem_limit(const void *kernel, size_t bytes);
+
+// Shape of one forward call, after validation.
+struct FwdShape {
+  int64_t T;
+  int d, d_i, r, bank, k;
+  int n_banks, d_s;
+  bool bf16;
+};
+
+// Scratch carve-up of the CUDA-core (gather) path.
+struct GatherPlan {
+  int tt_h;       // tokens per CTA of the h kernel
+  int tt_p;       // tokens per CTA of the logits/top-k kernel
+  int n_chunks;   // channel-slot chunks per token in the gather kernel
+  int chunk;      // slots per chunk
+  size_t off_h, off_idx, off_sig, off_part, off_mask, total;
+};
+GatherPlan plan_gather(const FwdShape &s);
+
+// Launchers (enqueue only; return cudaGetLastError()).
+cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
+                          cudaStream_t st);
+cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,
+                               float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
+                               cudaStream_t st);
+cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,
+                             int bank, int k, cudaStream_t st);
+cudaError_t launch_gather_ffn(const FwdShape &s, const GatherPlan &p, const void *x,
+                              const int *sel_idx, const float *sel_sig, const void *Wg,
+                              const void *Wu, const void *Wd, float *partial,
+                              cudaStream_t st);
+cudaError_t launch_reduce(const FwdShape &s, const GatherPlan &p, const float *partial,
+                          void *y, cudaStream_t st);
+
+}  // namespace sfn

@@ -125,3 +125,45 @@ def make_tokens(wl: Workload, T: int | None = None, seed: int = 0, layer: int = 
     else:
         raise ValueError(wl.x_dist)
     return _cast(x.astype(np.float32), wl)
+
+
+# ---------------------------------------------------------------------------
+# Device-side draws for benchmarking: the same distributions as above, drawn
+# with torch's CUDA generator (a different random stream, same recipe), so a
+# benchmark can hold many distinct layers without host generation time.
+
+def make_layer_device(wl: Workload, device, seed: int = 0, layer: int = 0) -> dict:
+    g = torch.Generator(device=device)
+    g.manual_seed(1_000_003 * seed + 7919 * layer + 17)
+
+    def draw(shape, std):
+        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+        return t.mul_(std).to(wl.torch_dtype)
+
+    A = draw((wl.r, wl.d), 1.0 / math.sqrt(wl.d))
+    B = draw((wl.d_i, wl.r), 1.0 / math.sqrt(wl.r))
+    Wg = draw((wl.d_i, wl.d), 1.0 / math.sqrt(wl.d))
+    Wu = draw((wl.d_i, wl.d), 1.0 / math.sqrt(wl.d))
+    Wd = draw((wl.d_i, wl.d), wl.wd_std)  # rows of W_down^T: i.i.d., so no transpose needed
+    return {"A": A, "B": B, "Wg": Wg, "Wu": Wu, "Wd": Wd}
+
+
+def make_tokens_device(wl: Workload, device, T: int | None = None, seed: int = 0,
+                       layer: int = 0) -> torch.Tensor:
+    T = wl.T if T is None else T
+    g = torch.Generator(device=device)
+    g.manual_seed(1_000_033 * seed + 104_729 * layer + 5)
+
+    def rms(z):
+        return z * torch.rsqrt(z.square().mean(dim=-1, keepdim=True) + 1e-6)
+
+    z = torch.randn((T, wl.d), generator=g, device=device, dtype=torch.float32)
+    if wl.x_dist == "normal":
+        x = z
+    elif wl.x_dist == "rmsnorm":
+        x = rms(z)
+    else:
+        U = torch.randn((wl.d, 32), generator=g, device=device) / math.sqrt(32)
+        c = torch.randn((T, 32), generator=g, device=device)
+        x = rms(z + 0.5 * c @ U.T)
+    return x.to(wl.torch_dtype)

@@ -1,0 +1,220 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Inputs come from the seeded generator (predictor_gated_channel_b200.inputs);
+expected values come only from the oracle.  Rules in tests/parity.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+import predictor_gated_channel_b200 as sfn
+from predictor_gated_channel_b200 import _capi
+from predictor_gated_channel_b200 import build as sfn_build
+from predictor_gated_channel_b200.inputs import WORKLOADS, make_layer, make_tokens
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    sfn_build.build()
+    _capi.lib()
+
+
+def _to_dev(layer):
+    return {k: v.to(DEV) for k, v in layer.items()}
+
+
+@pytest.fixture(scope="module")
+def full_layer():
+    """The full-width layer (d 4096, d_i 14336, r 448), bf16, seed 0."""
+    wl = WORKLOADS["decode"]
+    host = make_layer(wl)
+    return wl, host, _to_dev(host)
+
+
+def _run_forward(dev_layer, x_dev, bank, k):
+    y, mask = sfn.sparse_ffn_forward(x_dev, dev_layer["A"], dev_layer["B"], dev_layer["Wg"],
+                                     dev_layer["Wu"], dev_layer["Wd"], bank=bank, k=k)
+    torch.cuda.synchronize()
+    return y, mask
+
+
+def _check_forward(host, x_host, y, mask, bank, k, dtype, rows=None):
+    """Oracle on the (sampled) tokens; check mask rule and y error."""
+    if rows is None:
+        rows = np.arange(x_host.shape[0])
+    xs = x_host[torch.as_tensor(rows)]
+    logits = oracle.predict(xs, host["A"], host["B"])
+    gm = parity.to_u64(mask)[rows]
+    n_diff = parity.check_mask(gm, logits, bank, k)
+    y_ref = oracle.forward_given_mask(xs, logits, gm, host["Wg"], host["Wu"], host["Wd"], bank)
+    err = parity.y_error(y.float().cpu().numpy()[rows], y_ref)
+    assert err <= parity.Y_TOL[dtype], f"y error {err:.3g} > {parity.Y_TOL[dtype]}"
+    return n_diff, err
+
+
+# ------------------------------------------------------------------ bank top-k
+
+@pytest.mark.parametrize("bank,k", [(64, 16), (64, 1), (64, 63), (64, 64), (32, 5), (8, 3),
+                                    (1, 1), (48, 17)])
+def test_bank_topk_bit_exact_random(bank, k):
+    rng = np.random.default_rng(bank * 100 + k)
+    T, nb = 37, 29
+    p = rng.standard_normal((T, nb * bank)).astype(np.float32)
+    got = parity.to_u64(sfn.bank_topk(torch.from_numpy(p).to(DEV), bank, k))
+    torch.cuda.synchronize()
+    assert np.array_equal(got, oracle.bank_topk(p, bank, k))
+
+
+def test_bank_topk_bit_exact_adversarial():
+    rng = np.random.default_rng(7)
+    T, bank, k = 64, 64, 16
+    p = np.round(rng.standard_normal((T, 224 * bank)) * 2).astype(np.float32) / 2  # many ties
+    p[::3, ::5] = -0.0
+    p[1::3, ::7] = 0.0
+    p[2, :64] = np.nan
+    p[3, 5:40] = np.nan
+    p[4, :64] = np.inf
+    p[5, ::2] = -np.inf
+    p[6, :64] = 1.0                        # one value across the bank
+    p[7, :64] = np.float32(1e-45)          # denormals
+    p[8, 10:20] = np.finfo(np.float32).max
+    got = parity.to_u64(sfn.bank_topk(torch.from_numpy(p).to(DEV), bank, k))
+    torch.cuda.synchronize()
+    assert np.array_equal(got, oracle.bank_topk(p, bank, k))
+
+
+def test_bank_topk_oracle_logits_full_width(full_layer):
+    """Fed the oracle's own logits (rounded to fp32), the GPU mask is
+    bit-identical to the oracle's, at the full layer width."""
+    wl, host, _ = full_layer
+    x = make_tokens(WORKLOADS["prefill"], T=96)
+    logits = oracle.predict(x, host["A"], host["B"]).astype(np.float32)
+    got = parity.to_u64(sfn.bank_topk(torch.from_numpy(logits).to(DEV), 64, 16))
+    torch.cuda.synchronize()
+    assert np.array_equal(got, oracle.bank_topk(logits, 64, 16))
+
+
+# ------------------------------------------------------------------ predictor
+
+@pytest.mark.parametrize("name,T", [("tiny", 8), ("decode", 1), ("decode", 5), ("decode", 64)])
+def test_predict_logits(name, T, full_layer):
+    wl = WORKLOADS[name]
+    host = full_layer[1] if name != "tiny" else make_layer(wl)
+    x = make_tokens(wl, T=T)
+    got = sfn.predict(x.to(DEV), host["A"].to(DEV), host["B"].to(DEV))
+    torch.cuda.synchronize()
+    ref = oracle.predict(x, host["A"], host["B"])
+    err = np.abs(got.cpu().numpy().astype(np.float64) - ref).max()
+    assert err <= 1e-5 * np.abs(ref).max() + 1e-6, err
+
+
+# ------------------------------------------------------------------ forward
+
+def test_forward_tiny_f32():
+    wl = WORKLOADS["tiny"]
+    host = make_layer(wl)
+    x = make_tokens(wl)
+    y, mask = _run_forward(_to_dev(host), x.to(DEV), wl.bank, wl.k)
+    assert y.dtype == torch.float32
+    n_diff, err = _check_forward(host, x, y, mask, wl.bank, wl.k, "f32")
+    assert n_diff == 0
+
+
+@pytest.mark.parametrize("T", [1, 3, 17, 64])
+def test_forward_full_width_bf16(T, full_layer):
+    wl, host, dev = full_layer
+    x = make_tokens(wl, T=T, seed=T)
+    y, mask = _run_forward(dev, x.to(DEV), wl.bank, wl.k)
+    assert y.dtype == torch.bfloat16
+    _check_forward(host, x, y, mask, wl.bank, wl.k, "bf16")
+
+
+@pytest.mark.parametrize("bank,k", [(64, 1), (64, 63), (64, 64), (32, 8), (16, 16), (8, 3)])
+def test_forward_bank_k_variants_f32(bank, k):
+    wl = WORKLOADS["tiny"].with_(bank=bank, k=k)
+    host = make_layer(wl, seed=5)
+    x = make_tokens(wl, T=11, seed=5)
+    y, mask = _run_forward(_to_dev(host), x.to(DEV), bank, k)
+    _check_forward(host, x, y, mask, bank, k, "f32")
+
+
+def test_forward_dense_k64_equals_predictor_gated_dense(full_layer):
+    """k = bank keeps every channel (the recipe's predictor-gated dense FFN
+    stage): every mask word is all ones and y matches the oracle."""
+    wl, host, dev = full_layer
+    x = make_tokens(wl, T=2, seed=11)
+    y, mask = _run_forward(dev, x.to(DEV), 64, 64)
+    assert (parity.to_u64(mask) == np.uint64(2**64 - 1)).all()
+    _check_forward(host, x, y, mask, 64, 64, "bf16")
+
+
+@pytest.mark.parametrize("name", ["prefill", "long_prefill"])
+def test_forward_prefill_sampled(name, full_layer):
+    """Full prefill sizes in one call; the oracle checks 40 sampled tokens."""
+    wl = WORKLOADS[name]
+    _, host, dev = full_layer
+    x = make_tokens(wl)
+    y, mask = _run_forward(dev, x.to(DEV), wl.bank, wl.k)
+    rows = np.sort(np.random.default_rng(0).choice(wl.T, 40, replace=False))
+    rows[0], rows[-1] = 0, wl.T - 1
+    _check_forward(host, x, y, mask, wl.bank, wl.k, "bf16", rows=rows)
+    assert parity.popcount_ok(parity.to_u64(mask), wl.bank, wl.k)
+
+
+# ------------------------------------------------------------------ contract
+
+def test_workspace_variant_bit_identical_and_deterministic(full_layer):
+    wl, host, dev = full_layer
+    x = make_tokens(wl, T=9, seed=3).to(DEV)
+    y1, m1 = _run_forward(dev, x, 64, 16)
+    y2, m2 = _run_forward(dev, x, 64, 16)
+    nbytes = sfn.workspace_bytes(9, wl.d, wl.d_i, wl.r, 64, 16, torch.bfloat16)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    y3, m3 = sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"],
+                                    workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(m1, m2)
+    assert torch.equal(y1, y3) and torch.equal(m1, m3)
+
+
+def test_outputs_do_not_spill(full_layer):
+    """Canary words around y and mask stay untouched; mask may be omitted."""
+    wl, host, dev = full_layer
+    T = 5
+    x = make_tokens(wl, T=T, seed=9).to(DEV)
+    pad = 64
+    ybuf = torch.full((T * wl.d + 2 * pad,), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mbuf = torch.full((T * wl.n_banks + 2 * 8,), -12345, dtype=torch.int64, device=DEV)
+    y = ybuf[pad:pad + T * wl.d].view(T, wl.d)
+    m = mbuf[8:8 + T * wl.n_banks].view(T, wl.n_banks)
+    sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"], y=y, mask=m)
+    y_nomask, none = sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"],
+                                            dev["Wd"], want_mask=False)
+    torch.cuda.synchronize()
+    assert none is None
+    assert torch.isnan(ybuf[:pad].float()).all() and torch.isnan(ybuf[-pad:].float()).all()
+    assert (mbuf[:8] == -12345).all() and (mbuf[-8:] == -12345).all()
+    assert torch.equal(y, y_nomask)
+
+
+def test_launch_counter_counts_kernels(full_layer):
+    wl, host, dev = full_layer
+    x = make_tokens(wl, T=1).to(DEV)
+    c0 = sfn.kernel_launch_count()
+    _run_forward(dev, x, 64, 16)
+    assert sfn.kernel_launch_count() - c0 >= 3
+
+
+def test_zero_tokens(full_layer):
+    wl, host, dev = full_layer
+    x = torch.empty((0, wl.d), dtype=torch.bfloat16, device=DEV)
+    y, mask = _run_forward(dev, x, 64, 16)
+    assert y.shape == (0, wl.d) and mask.shape == (0, wl.n_banks)
