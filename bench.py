@@ -54,6 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--k", type=int, default=None, help="override top-k (e.g. 64: dense mask)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--settle", type=float, default=1.0,
+                    help="seconds of untimed load before timing (clock settling)")
     return ap.parse_args(argv)
 
 
@@ -292,7 +294,7 @@ def run_sfn(args, rank, world, local):
         for i in range(W % S):
             call(i, stream.cuda_stream)
         t_settle = time.time()
-        while time.time() - t_settle < 1.0:
+        while time.time() - t_settle < args.settle:
             g_full.replay()
         stream.synchronize()
 

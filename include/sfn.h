@@ -154,6 +154,39 @@ sfn_status sfn_sparse_ffn_forward_ws(const void *x, const void *A, const void *B
                                      int r, int bank, int k, void *workspace,
                                      size_t workspace_bytes, sfn_stream_t stream);
 
+/*
+ * The bf16 forward without any allocation.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory
+ * when they run the layer -- a plugin interface that hands the layer only
+ * its input and output pointers, a serving process whose allocator already
+ * owns the GPU's memory, or a latency-critical loop that must not risk
+ * cudaMalloc's implicit synchronisation.
+ *
+ * Arguments, layouts, results and checks are those of sfn_sparse_ffn_forward.
+ * The scratch is one fixed device array of SFN_STATIC_SCRATCH_BYTES inside
+ * the library, which the CUDA runtime keeps in the memory of every GPU that
+ * loads this library's code until the process exits.  The call allocates
+ * and frees nothing.
+ *   - A shape whose scratch need (sfn_workspace_bytes(..., SFN_DTYPE_BF16))
+ *     exceeds SFN_STATIC_SCRATCH_BYTES is rejected with SFN_ERR_WORKSPACE
+ *     before anything is enqueued.  For the 4096 x 14336 layer (r 448,
+ *     bank 64, k 16) every T up to 265 fits; sfn_workspace_bytes() tells
+ *     for any other shape.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call shares the one array per device.  Calls whose work overlaps
+ *     on the GPU (other streams, other host threads) race on it and produce
+ *     wrong results: serialise them.  The array keeps the previous call's
+ *     contents; each call writes every scratch byte before reading it, so
+ *     nothing needs clearing.
+ */
+#define SFN_STATIC_SCRATCH_BYTES (16u << 20)
+sfn_status sfn_sparse_ffn_forward_static(const void *x, const void *A, const void *B,
+                                         const void *Wg, const void *Wu, const void *Wd,
+                                         void *y, uint64_t *mask, int64_t T, int d, int d_i,
+                                         int r, int bank, int k, sfn_stream_t stream);
+
 /* float32 twins of the two forward entry points. */
 sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
                                       const float *Wg, const float *Wu, const float *Wd,

@@ -33,6 +33,7 @@ SIGNATURES = {
     "sfn_workspace_bytes": (_sz, [_i64, _ci, _ci, _ci, _ci, _ci, _ci]),
     "sfn_sparse_ffn_forward": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_ws": (_ci, _FWD + [_vp, _sz, _vp]),
+    "sfn_sparse_ffn_forward_static": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_f32": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_f32_ws": (_ci, _FWD + [_vp, _sz, _vp]),
     "sfn_timing_begin": (_ci, []),
@@ -40,6 +41,7 @@ SIGNATURES = {
     "sfn_stage_name": (ctypes.c_char_p, [_ci]),
 }
 SFN_STAGE_COUNT = 16
+SFN_STATIC_SCRATCH_BYTES = 16 << 20
 
 _lib = None
 _lock = threading.Lock()
