@@ -192,9 +192,10 @@ def stage_work(wl, T, union_channels):
         "pred_h": {"bytes": r * d * e + T * d * e + T * r * 4, "flops": 2 * T * d * r},
         "logits_topk": {"bytes": d_i * r * e + T * r * 4 + T * nb * 8 + T * d_s * 8,
                         "flops": 2 * T * r * d_i},
-        "gather_ffn": {"bytes": 3 * union_channels * d * e + T * d * e + T * d_s * 8,
-                       "flops": 6 * T * d_s * d},
-        "reduce": {"bytes": T * d * e, "flops": 0},
+        "gateup": {"bytes": 2 * union_channels * d * e + T * d * e + T * d_s * 12,
+                   "flops": 4 * T * d_s * d},
+        "down": {"bytes": union_channels * d * e + T * d_s * 8 + T * d * e,
+                 "flops": 2 * T * d_s * d},
     }
 
 

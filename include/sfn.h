@@ -211,12 +211,22 @@ sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const f
 enum {
   SFN_STAGE_PRED_H = 0,       /* h = A x                                */
   SFN_STAGE_LOGITS_TOPK = 1,  /* p = B h, bank top-k, sigma(p) of kept  */
-  SFN_STAGE_GATHER_FFN = 2,   /* kept gate/up rows, a_j, kept down rows */
-  SFN_STAGE_REDUCE = 3,       /* sum of partial output rows -> y        */
+  SFN_STAGE_GATEUP = 2,       /* kept gate/up rows -> a_j (few tokens)  */
+  SFN_STAGE_DOWN = 3,         /* kept down rows -> y (few tokens)       */
   SFN_STAGE_BANK_TOPK = 4,    /* standalone top-k on given logits       */
   SFN_STAGE_COUNT = 16        /* room for the stage ids of this library */
 };
 sfn_status sfn_timing_begin(void);
+
+/*
+ * Device error word of the current device (diagnostics; no counterpart in
+ * the paper).  Kernels never trap: a pipeline wait that gives up after about
+ * two seconds, or a failed index check, sets a bit here and the kernel
+ * returns early (its outputs are then invalid).  Bits: 1 = a bounded wait
+ * timed out, 2 = an index check failed.  This call synchronises the device,
+ * writes the word to *bits and, if `clear`, resets it to 0.
+ */
+sfn_status sfn_device_errors(unsigned *bits, int clear);
 sfn_status sfn_timing_end(double *ms, uint64_t *launches, int n);
 const char *sfn_stage_name(int stage);
 

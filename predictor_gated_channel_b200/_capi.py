@@ -37,6 +37,7 @@ SIGNATURES = {
     "sfn_sparse_ffn_forward_f32": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_f32_ws": (_ci, _FWD + [_vp, _sz, _vp]),
     "sfn_timing_begin": (_ci, []),
+    "sfn_device_errors": (_ci, [_vp, _ci]),
     "sfn_timing_end": (_ci, [_vp, _vp, _ci]),
     "sfn_stage_name": (ctypes.c_char_p, [_ci]),
 }

@@ -11,14 +11,15 @@
 
 namespace sfn {
 
+// The library's device error word (bits kDevErr*), set by kernels whose
+// bounded waits give up or whose index checks fail.
+__device__ unsigned g_sfn_device_error;
+
 namespace {
 std::atomic<uint64_t> g_launches{0};
 std::mutex g_dev_mu;
 DeviceInfo g_dev_cache[64];
 
-// CTAs the gather kernel aims for (two per SM of a 148-SM part); fixed so
-// that the scratch size does not depend on the device.
-constexpr int kGatherTargetCtas = 296;
 // Shape limits of the built kernels (shared-memory staging of x, h).
 constexpr int kMaxD = 16384;
 constexpr int kMaxR = 2048;
@@ -105,6 +106,9 @@ bool device_info(DeviceInfo *out) {
         cudaSuccess)
       return false;
     if (major != 10) return false;  // the library is built for sm_100a only
+    void *err = nullptr;
+    if (cudaGetSymbolAddress(&err, g_sfn_device_error) != cudaSuccess) return false;
+    c.err = static_cast<unsigned *>(err);
     c.num_sms = sms;
     c.max_smem_optin = smem;
     c.device = dev;
@@ -119,11 +123,6 @@ GatherPlan plan_gather(const FwdShape &s) {
   while (tt > 1 && (size_t)tt * s.d * sizeof(float) > kStageBudget) tt /= 2;
   p.tt_h = tt;
   p.tt_p = pow2_tokens(s.T, 8);
-  int64_t nc = (kGatherTargetCtas + s.T - 1) / s.T;
-  nc = std::min<int64_t>(nc, (s.d_s + 3) / 4);
-  nc = std::max<int64_t>(nc, 1);
-  p.chunk = (int)((s.d_s + nc - 1) / nc);
-  p.n_chunks = (s.d_s + p.chunk - 1) / p.chunk;
   size_t off = 0;
   p.off_h = off;
   off = align_up(off + (size_t)s.T * s.r * sizeof(float), 256);
@@ -131,9 +130,8 @@ GatherPlan plan_gather(const FwdShape &s) {
   off = align_up(off + (size_t)s.T * s.d_s * sizeof(int), 256);
   p.off_sig = off;
   off = align_up(off + (size_t)s.T * s.d_s * sizeof(float), 256);
-  p.off_part = off;
-  off = align_up(off + (size_t)s.T * p.n_chunks * s.d * sizeof(float), 256);
-  p.off_mask = off;
+  p.off_a = off;
+  off = align_up(off + (size_t)s.T * s.d_s * sizeof(float), 256);
   p.total = off;
   return p;
 }
@@ -199,7 +197,8 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
   float *h = nullptr;
   if (cudaMallocAsync((void **)&h, (size_t)T * r * sizeof(float), st) != cudaSuccess)
     return cuda_status(cudaErrorMemoryAllocation);
-  cudaError_t e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+  cudaError_t e = timed(SFN_STAGE_PRED_H, st,
+                        [&] { return launch_pred_h(s, p.tt_h, x, A, h, B, st); });
   if (e == cudaSuccess)
     e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
       return launch_logits_topk(s, p.tt_p, h, B, logits, nullptr, nullptr, nullptr, st);
@@ -235,19 +234,21 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
   float *h = reinterpret_cast<float *>(w + p.off_h);
   int *sel_idx = reinterpret_cast<int *>(w + p.off_idx);
   float *sel_sig = reinterpret_cast<float *>(w + p.off_sig);
-  float *partial = reinterpret_cast<float *>(w + p.off_part);
+  float *a_buf = reinterpret_cast<float *>(w + p.off_a);
+  const int gu_ctas = (int)std::min<int64_t>(dev.num_sms, (int64_t)T * s.d_s);
 
-  cudaError_t e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+  cudaError_t e = timed(SFN_STAGE_PRED_H, st,
+                        [&] { return launch_pred_h(s, p.tt_h, x, A, h, B, st); });
   if (e == cudaSuccess)
     e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
       return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, st);
     });
   if (e == cudaSuccess)
-    e = timed(SFN_STAGE_GATHER_FFN, st, [&] {
-      return launch_gather_ffn(s, p, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, st);
+    e = timed(SFN_STAGE_GATEUP, st, [&] {
+      return launch_gateup(s, gu_ctas, x, sel_idx, sel_sig, Wg, Wu, Wd, a_buf, dev.err, st);
     });
   if (e == cudaSuccess)
-    e = timed(SFN_STAGE_REDUCE, st, [&] { return launch_reduce(s, p, partial, y, st); });
+    e = timed(SFN_STAGE_DOWN, st, [&] { return launch_down(s, sel_idx, a_buf, Wd, y, st); });
   if (own_ws) {
     cudaError_t ef = cudaFreeAsync(ws, st);
     if (e == cudaSuccess) e = ef;
@@ -381,12 +382,24 @@ sfn_status sfn_timing_end(double *ms, uint64_t *launches, int n) {
   return st;
 }
 
+sfn_status sfn_device_errors(unsigned *bits, int clear) {
+  DeviceInfo dev;
+  if (!device_info(&dev)) return SFN_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, dev.err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_status(cudaErrorUnknown);
+  if (clear && v != 0 && cudaMemset(dev.err, 0, sizeof v) != cudaSuccess)
+    return cuda_status(cudaErrorUnknown);
+  if (bits) *bits = v;
+  return SFN_OK;
+}
+
 const char *sfn_stage_name(int stage) {
   switch (stage) {
     case SFN_STAGE_PRED_H: return "pred_h";
     case SFN_STAGE_LOGITS_TOPK: return "logits_topk";
-    case SFN_STAGE_GATHER_FFN: return "gather_ffn";
-    case SFN_STAGE_REDUCE: return "reduce";
+    case SFN_STAGE_GATEUP: return "gateup";
+    case SFN_STAGE_DOWN: return "down";
     case SFN_STAGE_BANK_TOPK: return "bank_topk";
   }
   return "unused";

@@ -1,17 +1,23 @@
-// predict_topk.cu -- CUDA-core kernels of the predictor and the bank top-k.
+// predict_topk.cu -- CUDA-core kernels of the predictor and the bank top-k
+// (the few-token path, and the standalone top-k).
 //
 // Predictor "R^d -> R^448 -> R^{d_i}" and the bank-wise hard top-16 of 64:
 // "Continual LLM Upcycling: A Predictor-Gated Bank-Wise Sparsity Training
 // Recipe for Dense-to-Sparse LLMs", gist.science summary, "1. Architectuur".
 //
-//   k_pred_h       h[t] = A x[t]                (fp32 out, one warp per row of A)
+//   k_pred_h       h[t] = A x[t] (fp32), one warp per row of A with the whole
+//                  row's 16-byte loads in flight; token groups of TT share
+//                  each row load.  The first token group also issues L2
+//                  prefetches of B, so that k_logits_topk reads B from L2.
 //   k_logits_topk  p[t] = B h[t] for one bank, then (optionally) that bank's
 //                  top-k: mask word, kept channel ids and sigma(p) in
 //                  ascending channel order (one CTA per bank and token group)
 //   k_bank_topk    standalone top-k on float32 logits (one warp per bank)
 //
-// Every weight element is read with 16-byte loads; accumulation is fp32 in a
-// fixed order.
+// Both chained kernels use programmatic dependent launch: they let the next
+// kernel start early, issue only L2 prefetches of weights before
+// griddepcontrol.wait, and touch every other buffer after it.
+#include "async_util.cuh"
 #include "sfn_internal.cuh"
 
 namespace sfn {
@@ -46,36 +52,65 @@ __device__ __forceinline__ void stage_rows(float *xs, const char *x, int64_t t0,
 
 // h[t][m] = sum_n A[m][n] x[t][n].  1-D grid over (token group, row block):
 // blockIdx.x = token_group * ceil(r / kWarps) + row_block.
+// If Bpf != nullptr, the CTAs of token group 0 prefetch B (Bpf_bytes) to L2.
 template <class E, int TT>
 __global__ void __launch_bounds__(kThreads) k_pred_h(const char *__restrict__ x,
                                                      const char *__restrict__ A,
                                                      float *__restrict__ h, int64_t T, int d,
-                                                     int r) {
+                                                     int r, const char *__restrict__ Bpf,
+                                                     int64_t Bpf_bytes) {
   extern __shared__ float4 smem_f4[];
   float *xs = reinterpret_cast<float *>(smem_f4);
   const int row_blocks = (r + kWarps - 1) / kWarps;
-  const int64_t t0 = (int64_t)(blockIdx.x / row_blocks) * TT;
+  const int64_t tg = blockIdx.x / row_blocks;
+  const int rb = blockIdx.x % row_blocks;
+  pdl_launch_dependents();
+  if (Bpf != nullptr && tg == 0 && threadIdx.x == 0) {
+    // this CTA's 16-byte-aligned share of B
+    const int64_t share = ((Bpf_bytes + row_blocks - 1) / row_blocks + 15) / 16 * 16;
+    const int64_t beg = rb * share;
+    const int64_t end = beg + share < Bpf_bytes ? beg + share : Bpf_bytes;
+    for (int64_t o = beg; o < end; o += 65536) {
+      const int64_t n = end - o < 65536 ? end - o : 65536;
+      prefetch_l2(Bpf + o, (uint32_t)n);
+    }
+  }
+  pdl_wait();
+
+  const int64_t t0 = tg * TT;
   const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
   stage_rows<E, TT>(xs, x, t0, nt, d);
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = (blockIdx.x % row_blocks) * kWarps + warp;
+  const int m = rb * kWarps + warp;
   if (m >= r) return;
   const int nchunk = d / E::kVec;
   const char *row = A + (int64_t)m * d * E::kBytes;
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-#pragma unroll 4
-  for (int c = lane; c < nchunk; c += 32) {
-    float a[E::kVec];
-    E::unpack(ld_stream16(row + (int64_t)c * 16), a);
+  // 16 loads per lane in flight (a whole 8 KB bf16 row per warp)
+  for (int c0 = lane; c0 < nchunk; c0 += 32 * 16) {
+    uint4 v[16];
 #pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const float *xr = xs + t * d + c * E::kVec;
+    for (int u = 0; u < 16; ++u) {
+      const int c = c0 + 32 * u;
+      v[u] = (c < nchunk) ? ld_stream16(row + (int64_t)c * 16) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int e = 0; e < E::kVec; ++e) acc[t] = fmaf(a[e], xr[e], acc[t]);
+    for (int u = 0; u < 16; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nchunk) {
+        float a[E::kVec];
+        E::unpack(v[u], a);
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          const float *xr = xs + t * d + c * E::kVec;
+#pragma unroll
+          for (int e = 0; e < E::kVec; ++e) acc[t] = fmaf(a[e], xr[e], acc[t]);
+        }
+      }
     }
   }
 #pragma unroll
@@ -103,6 +138,8 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
   const int b = blockIdx.x % n_banks;
   const int64_t t0 = (int64_t)(blockIdx.x / n_banks) * TT;
   const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
+  pdl_launch_dependents();
+  pdl_wait();
   for (int i = threadIdx.x; i < TT * r; i += blockDim.x) {
     const int t = i / r;
     hs[i] = (t < nt) ? h[(t0 + t) * r + (i - t * r)] : 0.f;
@@ -111,28 +148,55 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunk = r / E::kVec;
-  for (int jl = warp; jl < bank; jl += kWarps) {
-    const int j = b * bank + jl;
-    const char *row = B + (int64_t)j * r * E::kBytes;
-    float acc[TT];
+  // Each warp owns rows jl = warp + kWarps * i; a group of 4 rows x 2 chunk
+  // columns of loads is issued before any arithmetic.
+  for (int jl0 = warp; jl0 < bank; jl0 += 4 * kWarps) {
+    float acc[4][TT];
 #pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-    for (int c = lane; c < nchunk; c += 32) {
-      float w[E::kVec];
-      E::unpack(ld_stream16(row + (int64_t)c * 16), w);
+    for (int q = 0; q < 4; ++q)
 #pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        const float *hr = hs + t * r + c * E::kVec;
+      for (int t = 0; t < TT; ++t) acc[q][t] = 0.f;
+    for (int c0 = lane; c0 < nchunk; c0 += 64) {
+      uint4 v[4][2];
 #pragma unroll
-        for (int e = 0; e < E::kVec; ++e) acc[t] = fmaf(w[e], hr[e], acc[t]);
+      for (int q = 0; q < 4; ++q) {
+        const int jl = jl0 + q * kWarps;
+        const char *row = B + (int64_t)(b * bank + jl) * r * E::kBytes;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = c0 + 32 * u;
+          v[q][u] = (jl < bank && c < nchunk) ? ld_nc16(row + (int64_t)c * 16)
+                                              : make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = c0 + 32 * u;
+          if (c < nchunk) {
+            float w[E::kVec];
+            E::unpack(v[q][u], w);
+#pragma unroll
+            for (int t = 0; t < TT; ++t) {
+              const float *hr = hs + t * r + c * E::kVec;
+#pragma unroll
+              for (int e = 0; e < E::kVec; ++e) acc[q][t] = fmaf(w[e], hr[e], acc[q][t]);
+            }
+          }
+        }
       }
     }
 #pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const float v = warp_sum(acc[t]);
-      if (lane == 0) {
-        ps[t * 64 + jl] = v;
-        if (kWriteLogits && t < nt) logits[(t0 + t) * d_i + j] = v;
+    for (int q = 0; q < 4; ++q) {
+      const int jl = jl0 + q * kWarps;
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const float v = warp_sum(acc[q][t]);
+        if (lane == 0 && jl < bank) {
+          ps[t * 64 + jl] = v;
+          if (kWriteLogits && t < nt) logits[(t0 + t) * d_i + b * bank + jl] = v;
+        }
       }
     }
   }
@@ -153,7 +217,7 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
       idx_row[s] = b * bank + lane;
       sig_row[s] = sigmoid_f32(p0);
     }
-    if (lane + 32 < 64 && ((word >> (lane + 32)) & 1ull)) {
+    if ((word >> (lane + 32)) & 1ull) {
       const int s = __popcll(word & ((1ull << (lane + 32)) - 1ull));
       idx_row[s] = b * bank + lane + 32;
       sig_row[s] = sigmoid_f32(p1);
@@ -175,23 +239,20 @@ __global__ void __launch_bounds__(kThreads) k_bank_topk(const float *__restrict_
   if (lane == 0) mask[wi] = word;
 }
 
-template <class K>
-cudaError_t set_smem(K kernel, size_t bytes) {
-  return ensure_smem_limit(reinterpret_cast<const void *>(kernel), bytes);
-}
-
 template <class E, int TT>
 cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, float *h,
-                      cudaStream_t st) {
+                      const void *Bpf, cudaStream_t st) {
   const size_t smem = (size_t)TT * s.d * sizeof(float);
   auto kern = k_pred_h<E, TT>;
-  cudaError_t e = set_smem(kern, smem);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)((s.r + kWarps - 1) / kWarps) * ((s.T + TT - 1) / TT);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<(unsigned)blocks, kThreads, smem, st>>>((const char *)x, (const char *)A, h, s.T, s.d, s.r);
+  const int64_t bpf_bytes = (int64_t)s.d_i * s.r * (s.bf16 ? 2 : 4);
+  e = launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreads), smem, st, (const char *)x,
+                 (const char *)A, h, s.T, s.d, s.r, (const char *)Bpf, bpf_bytes);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 template <class E, int TT, bool W, bool K>
@@ -199,14 +260,14 @@ cudaError_t logits_tt(const FwdShape &s, const float *h, const void *B, float *l
                       uint64_t *mask, int *sel_idx, float *sel_sig, cudaStream_t st) {
   const size_t smem = (size_t)TT * (s.r + 64) * sizeof(float);
   auto kern = k_logits_topk<E, TT, W, K>;
-  cudaError_t e = set_smem(kern, smem);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)s.n_banks * ((s.T + TT - 1) / TT);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<(unsigned)blocks, kThreads, smem, st>>>(h, (const char *)B, logits, mask, sel_idx, sel_sig, s.T,
-                                     s.d_i, s.r, s.bank, s.k);
+  e = launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreads), smem, st, h, (const char *)B,
+                 logits, mask, sel_idx, sel_sig, s.T, s.d_i, s.r, s.bank, s.k);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 template <class E, bool W, bool K>
@@ -224,20 +285,20 @@ cudaError_t logits_dispatch(const FwdShape &s, int tt, const float *h, const voi
 }  // namespace
 
 cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
-                          cudaStream_t st) {
+                          const void *Bpf, cudaStream_t st) {
   if (s.bf16) {
     switch (tt) {
-      case 1: return pred_h_tt<EltBF16, 1>(s, x, A, h, st);
-      case 2: return pred_h_tt<EltBF16, 2>(s, x, A, h, st);
-      case 4: return pred_h_tt<EltBF16, 4>(s, x, A, h, st);
-      default: return pred_h_tt<EltBF16, 8>(s, x, A, h, st);
+      case 1: return pred_h_tt<EltBF16, 1>(s, x, A, h, Bpf, st);
+      case 2: return pred_h_tt<EltBF16, 2>(s, x, A, h, Bpf, st);
+      case 4: return pred_h_tt<EltBF16, 4>(s, x, A, h, Bpf, st);
+      default: return pred_h_tt<EltBF16, 8>(s, x, A, h, Bpf, st);
     }
   }
   switch (tt) {
-    case 1: return pred_h_tt<EltF32, 1>(s, x, A, h, st);
-    case 2: return pred_h_tt<EltF32, 2>(s, x, A, h, st);
-    case 4: return pred_h_tt<EltF32, 4>(s, x, A, h, st);
-    default: return pred_h_tt<EltF32, 8>(s, x, A, h, st);
+    case 1: return pred_h_tt<EltF32, 1>(s, x, A, h, Bpf, st);
+    case 2: return pred_h_tt<EltF32, 2>(s, x, A, h, Bpf, st);
+    case 4: return pred_h_tt<EltF32, 4>(s, x, A, h, Bpf, st);
+    default: return pred_h_tt<EltF32, 8>(s, x, A, h, Bpf, st);
   }
 }
 

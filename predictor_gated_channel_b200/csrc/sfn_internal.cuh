@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "sfn.h"
 
 namespace sfn {
@@ -111,6 +113,7 @@ struct DeviceInfo {
   int device = -1;
   int num_sms = 0;
   int max_smem_optin = 0;
+  unsigned *err = nullptr;  // device address of the library's error word
 };
 // Cached per-device properties; returns false if no device is usable.
 bool device_info(DeviceInfo *out);
@@ -135,27 +138,44 @@ struct FwdShape {
 
 // Scratch carve-up of the CUDA-core (gather) path.
 struct GatherPlan {
-  int tt_h;       // tokens per CTA of the h kernel
-  int tt_p;       // tokens per CTA of the logits/top-k kernel
-  int n_chunks;   // channel-slot chunks per token in the gather kernel
-  int chunk;      // slots per chunk
-  size_t off_h, off_idx, off_sig, off_part, off_mask, total;
+  int tt_h;  // tokens per CTA of the h kernel
+  int tt_p;  // tokens per CTA of the logits/top-k kernel
+  size_t off_h, off_idx, off_sig, off_a, total;
 };
 GatherPlan plan_gather(const FwdShape &s);
 
-// Launchers (enqueue only; return cudaGetLastError()).
+// Launch with programmatic stream serialisation (programmatic dependent
+// launch): the kernel may start while its predecessor in the stream is still
+// running and must call griddepcontrol.wait before touching its outputs.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Launchers (enqueue only; return the launch status).
 cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
-                          cudaStream_t st);
+                          const void *Bpf, cudaStream_t st);
 cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,
                                float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
                                cudaStream_t st);
 cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,
                              int bank, int k, cudaStream_t st);
-cudaError_t launch_gather_ffn(const FwdShape &s, const GatherPlan &p, const void *x,
-                              const int *sel_idx, const float *sel_sig, const void *Wg,
-                              const void *Wu, const void *Wd, float *partial,
-                              cudaStream_t st);
-cudaError_t launch_reduce(const FwdShape &s, const GatherPlan &p, const float *partial,
-                          void *y, cudaStream_t st);
+size_t gateup_smem_bytes(const FwdShape &s);
+cudaError_t launch_gateup(const FwdShape &s, int ctas, const void *x, const int *sel_idx,
+                          const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
+                          float *a_out, unsigned *err, cudaStream_t st);
+cudaError_t launch_down(const FwdShape &s, const int *sel_idx, const float *a, const void *Wd,
+                        void *y, cudaStream_t st);
 
 }  // namespace sfn

@@ -25,3 +25,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors(request):
+    """After every GPU test: the library's device error word must be clear
+    (no bounded wait gave up, no index check failed)."""
+    yield
+    if "gpu" not in request.keywords:
+        return
+    import ctypes
+    from predictor_gated_channel_b200 import _capi
+    bits = ctypes.c_uint(0)
+    assert _capi.lib().sfn_device_errors(ctypes.byref(bits), 1) == _capi.SFN_OK
+    assert bits.value == 0, f"device error word {bits.value:#x}"
