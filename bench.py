@@ -185,17 +185,23 @@ def stage_work(wl, T, union_channels):
     """Algorithmic bytes and useful FLOPs of each stage for one call on T tokens.
 
     union_channels: number of distinct kept channels over the T tokens (the
-    rows of Wg, Wu, Wd that must be read at least once)."""
+    rows of Wg, Wu, Wd that must be read at least once).  Tensor-core stages
+    count the same useful work; their dense tiles do more arithmetic."""
     e = 2 if wl.dtype == "bf16" else 4
     d, d_i, r, d_s, nb = wl.d, wl.d_i, wl.r, wl.d_s, wl.n_banks
+    pred_h = {"bytes": r * d * e + T * d * e + T * r * 4, "flops": 2 * T * d * r}
+    logits = {"bytes": d_i * r * e + T * r * 4 + T * nb * 8 + T * d_s * 8,
+              "flops": 2 * T * r * d_i}
+    ffn = {"bytes": 3 * union_channels * d * e + T * d * e + T * d_s * 8,
+           "flops": 6 * T * d_s * d}
     return {
-        "pred_h": {"bytes": r * d * e + T * d * e + T * r * 4, "flops": 2 * T * d * r},
-        "logits_topk": {"bytes": d_i * r * e + T * r * 4 + T * nb * 8 + T * d_s * 8,
-                        "flops": 2 * T * r * d_i},
-        "gateup": {"bytes": 2 * union_channels * d * e + T * d * e + T * d_s * 12,
-                   "flops": 4 * T * d_s * d},
-        "down": {"bytes": union_channels * d * e + T * d_s * 8 + T * d * e,
-                 "flops": 2 * T * d_s * d},
+        "pred_h": pred_h, "logits_topk": logits, "ffn": ffn,
+        "reduce": {"bytes": T * d * e, "flops": 0},
+        "tc_h": pred_h, "tc_logits_topk": logits,
+        "tc_gateup": {"bytes": 2 * union_channels * d * e + T * d * e + T * d_i * e,
+                      "flops": 4 * T * d_s * d},
+        "tc_down": {"bytes": union_channels * d * e + T * d_i * e + T * d * e,
+                    "flops": 2 * T * d_s * d},
     }
 
 
@@ -348,7 +354,7 @@ def run_sfn(args, rank, world, local):
     for v in stages.values():
         v["share"] = v["ms_total"] / tot
     work = stage_work(wl, T, union)
-    bound = "hbm" if T <= 64 else "tensor"
+    bound = "hbm" if T <= 256 else "tensor"
     dom = max(stages, key=lambda n: stages[n]["ms_total"])
     dom_s = stages[dom]["us_per_launch"] * 1e-6
     if bound == "hbm":
@@ -409,7 +415,8 @@ def run_sfn(args, rank, world, local):
         return None
 
     value = world * T * K / (elapsed_ms_max * 1e-3)
-    step_bytes = sum(work[n]["bytes"] for n in work)
+    # the path's algorithmic minimum: predictor weights, kept rows, x and y
+    step_bytes = sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "ffn", "reduce"))
     step_flops = T * useful_flops_per_token(wl)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,

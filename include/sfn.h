@@ -83,7 +83,10 @@ typedef enum sfn_status {
   SFN_ERR_MISALIGNED = 2,    /* a pointer not 16-byte aligned, or d or r not
                                 a multiple of 16 bytes of its element type */
   SFN_ERR_UNSUPPORTED = 3,   /* a valid shape outside the built kernels'
-                                limits (d > 16384, r > 2048, d_i > 2^24) */
+                                limits: d > 8192, r > 2048, d_i > 2^24;
+                                on the CUDA-core path also d not a
+                                multiple of 64 (bf16) / 32 (f32), or
+                                d > 4096 for f32 */
   SFN_ERR_WORKSPACE = 4,     /* *_ws scratch NULL, misaligned or smaller than
                                 sfn_workspace_bytes() */
   SFN_ERR_CUDA = 5           /* a CUDA runtime call or launch failed */
@@ -187,6 +190,34 @@ sfn_status sfn_sparse_ffn_forward_static(const void *x, const void *A, const voi
                                          void *y, uint64_t *mask, int64_t T, int d, int d_i,
                                          int r, int bank, int k, sfn_stream_t stream);
 
+/*
+ * Which kernels compute the forward.  The result is the same either way
+ * (within rounding; the mask may differ only at exact-threshold ties of the
+ * differently rounded logits).
+ *   SFN_PATH_CUDA_CORE  gather kernels that read only the kept rows (few
+ *                       tokens: every T, any bank <= 64, bf16 or f32);
+ *   SFN_PATH_TENSOR     tcgen05 tensor-core GEMMs over 128-token tiles with
+ *                       the top-k and the sigma(p) g u mask fused into their
+ *                       epilogues (bf16, bank 64, d and d_i multiples of
+ *                       256, r a multiple of 64 up to 512);
+ *   SFN_PATH_AUTO       the tensor path from T >= 1024 when the shape allows
+ *                       it, the CUDA-core path otherwise.
+ */
+typedef enum sfn_path {
+  SFN_PATH_AUTO = 0,
+  SFN_PATH_CUDA_CORE = 1,
+  SFN_PATH_TENSOR = 2
+} sfn_path;
+
+/* sfn_sparse_ffn_forward_ws with an explicit path.  SFN_PATH_TENSOR on a
+ * shape the tensor path does not cover returns SFN_ERR_UNSUPPORTED.
+ * sfn_workspace_bytes() covers both paths. */
+sfn_status sfn_sparse_ffn_forward_path(const void *x, const void *A, const void *B,
+                                       const void *Wg, const void *Wu, const void *Wd,
+                                       void *y, uint64_t *mask, int64_t T, int d, int d_i,
+                                       int r, int bank, int k, sfn_path path, void *workspace,
+                                       size_t workspace_bytes, sfn_stream_t stream);
+
 /* float32 twins of the two forward entry points. */
 sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
                                       const float *Wg, const float *Wu, const float *Wd,
@@ -211,9 +242,13 @@ sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const f
 enum {
   SFN_STAGE_PRED_H = 0,       /* h = A x                                */
   SFN_STAGE_LOGITS_TOPK = 1,  /* p = B h, bank top-k, sigma(p) of kept  */
-  SFN_STAGE_GATEUP = 2,       /* kept gate/up rows -> a_j (few tokens)  */
-  SFN_STAGE_DOWN = 3,         /* kept down rows -> y (few tokens)       */
+  SFN_STAGE_FFN = 2,          /* kept gate/up/down rows -> partial y    */
+  SFN_STAGE_REDUCE = 3,       /* partial rows -> y (few tokens)         */
   SFN_STAGE_BANK_TOPK = 4,    /* standalone top-k on given logits       */
+  SFN_STAGE_TC_H = 5,         /* tensor cores: h = A x, split hi/lo     */
+  SFN_STAGE_TC_LOGITS_TOPK = 6, /* tensor cores: logits + fused top-k   */
+  SFN_STAGE_TC_GATEUP = 7,    /* tensor cores: masked sigma(p) g u      */
+  SFN_STAGE_TC_DOWN = 8,      /* tensor cores: y = act W_down           */
   SFN_STAGE_COUNT = 16        /* room for the stage ids of this library */
 };
 sfn_status sfn_timing_begin(void);

@@ -94,13 +94,21 @@ def bank_topk(logits, bank: int = 64, k: int = 16, out=None, stream=None):
     return out
 
 
+PATHS = {"auto": _capi.SFN_PATH_AUTO, "cuda_core": _capi.SFN_PATH_CUDA_CORE,
+         "tensor": _capi.SFN_PATH_TENSOR}
+
+
 def sparse_ffn_forward(x, A, B, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None, mask=None,
-                       workspace=None, want_mask: bool = True, stream=None):
+                       workspace=None, want_mask: bool = True, path: str = "auto",
+                       stream=None):
     """The sparse FFN forward.  Wd is channel-major: Wd[j] = W_down[:, j].
 
     Returns (y [T, d] in x's dtype, mask int64 [T, d_i/bank] or None).  With
     ``workspace`` (a uint8 CUDA tensor of at least ``workspace_bytes(...)``)
     the call uses it as scratch instead of allocating stream-ordered memory.
+    ``path`` ("auto", "cuda_core" or "tensor") picks the kernels; a bf16
+    call with an explicit path always uses caller scratch (allocated here
+    when ``workspace`` is None).
     """
     torch = _torch()
     names = ("x", "A", "B", "Wg", "Wu", "Wd")
@@ -130,6 +138,17 @@ def sparse_ffn_forward(x, A, B, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None,
     L = _capi.lib()
     args = [x.data_ptr(), A.data_ptr(), B.data_ptr(), Wg.data_ptr(), Wu.data_ptr(),
             Wd.data_ptr(), y.data_ptr(), mptr, T, d, d_i, r, bank, k]
+    if path != "auto":
+        if elt != _capi.SFN_DTYPE_BF16:
+            raise ValueError("an explicit path is available for bf16 only")
+        if workspace is None:
+            nbytes = workspace_bytes(T, d, d_i, r, bank, k, x.dtype)
+            workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        _dev(workspace, "workspace")
+        _capi.check(L.sfn_sparse_ffn_forward_path(
+            *args, PATHS[path], workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), st), "sfn_sparse_ffn_forward_path")
+        return y, mask
     if workspace is None:
         fn = (L.sfn_sparse_ffn_forward if elt == _capi.SFN_DTYPE_BF16
               else L.sfn_sparse_ffn_forward_f32)

@@ -17,6 +17,10 @@ SFN_ERR_UNSUPPORTED = 3
 SFN_ERR_WORKSPACE = 4
 SFN_ERR_CUDA = 5
 
+SFN_PATH_AUTO = 0
+SFN_PATH_CUDA_CORE = 1
+SFN_PATH_TENSOR = 2
+
 SFN_DTYPE_BF16 = 0
 SFN_DTYPE_F32 = 1
 
@@ -34,6 +38,7 @@ SIGNATURES = {
     "sfn_sparse_ffn_forward": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_ws": (_ci, _FWD + [_vp, _sz, _vp]),
     "sfn_sparse_ffn_forward_static": (_ci, _FWD + [_vp]),
+    "sfn_sparse_ffn_forward_path": (_ci, _FWD + [_ci, _vp, _sz, _vp]),
     "sfn_sparse_ffn_forward_f32": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_f32_ws": (_ci, _FWD + [_vp, _sz, _vp]),
     "sfn_timing_begin": (_ci, []),

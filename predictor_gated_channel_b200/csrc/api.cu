@@ -21,10 +21,14 @@ std::mutex g_dev_mu;
 DeviceInfo g_dev_cache[64];
 
 // Shape limits of the built kernels (shared-memory staging of x, h).
-constexpr int kMaxD = 16384;
+constexpr int kMaxD = 8192;
 constexpr int kMaxR = 2048;
 constexpr int kMaxDi = 1 << 24;
 constexpr size_t kStageBudget = 96 * 1024;  // bytes of x rows staged per CTA
+// The few-token gate/up/down kernel spreads each token over this many CTAs
+// (divided among the tokens); fixed so the scratch size does not depend on
+// the device.  148 = the SM count of a B200.
+constexpr int kPlanSms = 148;
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
@@ -123,6 +127,7 @@ GatherPlan plan_gather(const FwdShape &s) {
   while (tt > 1 && (size_t)tt * s.d * sizeof(float) > kStageBudget) tt /= 2;
   p.tt_h = tt;
   p.tt_p = pow2_tokens(s.T, 8);
+  p.cpt = ffn_ctas_per_token(s, kPlanSms);
   size_t off = 0;
   p.off_h = off;
   off = align_up(off + (size_t)s.T * s.r * sizeof(float), 256);
@@ -130,8 +135,8 @@ GatherPlan plan_gather(const FwdShape &s) {
   off = align_up(off + (size_t)s.T * s.d_s * sizeof(int), 256);
   p.off_sig = off;
   off = align_up(off + (size_t)s.T * s.d_s * sizeof(float), 256);
-  p.off_a = off;
-  off = align_up(off + (size_t)s.T * s.d_s * sizeof(float), 256);
+  p.off_part = off;
+  off = align_up(off + (size_t)s.T * p.cpt * s.d * sizeof(float), 256);
   p.total = off;
   return p;
 }
@@ -188,32 +193,61 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
   if ((s0 = check_rows(d, r, bf16)) != SFN_OK) return s0;
   if (T == 0) return SFN_OK;
   if (!x || !A || !B || !logits) return SFN_ERR_INVALID_VALUE;
-  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(logits, 4))
+  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(logits, 16))
     return SFN_ERR_MISALIGNED;
   DeviceInfo dev;
   if (!device_info(&dev)) return SFN_ERR_CUDA;
-  FwdShape s = make_shape(T, d, d_i, r, 1, 1, bf16);
-  GatherPlan p = plan_gather(s);
-  float *h = nullptr;
-  if (cudaMallocAsync((void **)&h, (size_t)T * r * sizeof(float), st) != cudaSuccess)
+  FwdShape s = make_shape(T, d, d_i, r, 64, 16, bf16);
+  const bool tc = tc_shape_ok(s) && T >= 1024;
+  const size_t need = tc ? (size_t)T * 2 * r * 2 : (size_t)T * r * sizeof(float);
+  void *scratch = nullptr;
+  if (cudaMallocAsync(&scratch, need, st) != cudaSuccess)
     return cuda_status(cudaErrorMemoryAllocation);
-  cudaError_t e = timed(SFN_STAGE_PRED_H, st,
-                        [&] { return launch_pred_h(s, p.tt_h, x, A, h, B, st); });
-  if (e == cudaSuccess)
-    e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
-      return launch_logits_topk(s, p.tt_p, h, B, logits, nullptr, nullptr, nullptr, st);
-    });
-  cudaError_t ef = cudaFreeAsync(h, st);
+  cudaError_t e;
+  if (tc) {
+    uint16_t *h2 = static_cast<uint16_t *>(scratch);
+    e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, st); });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
+                [&] { return launch_tc_logits(s, dev, h2, B, logits, nullptr, nullptr, st); });
+  } else {
+    GatherPlan p = plan_gather(s);
+    float *h = static_cast<float *>(scratch);
+    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
+        return launch_logits_topk(s, p.tt_p, h, B, logits, nullptr, nullptr, nullptr, dev.err,
+                                  st);
+      });
+  }
+  cudaError_t ef = cudaFreeAsync(scratch, st);
   if (e == cudaSuccess) e = ef;
   return cuda_status(e);
 }
 
+// Fewest tokens for which the automatic choice takes the tensor-core path.
+constexpr int64_t kTcMinTokens = 1024;
+
+bool use_tensor_path(const FwdShape &s, sfn_path path) {
+  if (path == SFN_PATH_CUDA_CORE) return false;
+  if (!tc_shape_ok(s)) return false;
+  return path == SFN_PATH_TENSOR || s.T >= kTcMinTokens;
+}
+
+size_t workspace_for(const FwdShape &s) {
+  size_t need = plan_gather(s).total;
+  if (tc_shape_ok(s)) need = std::max(need, plan_tc(s).total);
+  return need;
+}
+
 sfn_status forward_impl(const void *x, const void *A, const void *B, const void *Wg,
                         const void *Wu, const void *Wd, void *y, uint64_t *mask, int64_t T,
-                        int d, int d_i, int r, int bank, int k, bool bf16, void *ws,
-                        size_t ws_bytes, bool own_ws, cudaStream_t st) {
+                        int d, int d_i, int r, int bank, int k, bool bf16, sfn_path path,
+                        void *ws, size_t ws_bytes, bool own_ws, cudaStream_t st) {
   sfn_status s0 = check_shape(T, d, d_i, r, bank, k);
   if (s0 != SFN_OK) return s0;
+  if (path != SFN_PATH_AUTO && path != SFN_PATH_CUDA_CORE && path != SFN_PATH_TENSOR)
+    return SFN_ERR_INVALID_VALUE;
   if ((s0 = check_limits(d, d_i, r)) != SFN_OK) return s0;
   if ((s0 = check_rows(d, r, bf16)) != SFN_OK) return s0;
   if (T == 0) return SFN_OK;
@@ -223,32 +257,52 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
       (mask && !aligned(mask, 8)))
     return SFN_ERR_MISALIGNED;
   FwdShape s = make_shape(T, d, d_i, r, bank, k, bf16);
-  GatherPlan p = plan_gather(s);
-  if (!own_ws && (ws == nullptr || !aligned(ws, 256) || ws_bytes < p.total))
+  if (path == SFN_PATH_TENSOR && !tc_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
+  const bool tc = use_tensor_path(s, path);
+  if (!tc && !ffn_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
+  const size_t need = tc ? plan_tc(s).total : plan_gather(s).total;
+  if (!own_ws && (ws == nullptr || !aligned(ws, 256) || ws_bytes < need))
     return SFN_ERR_WORKSPACE;
   DeviceInfo dev;
   if (!device_info(&dev)) return SFN_ERR_CUDA;
-  if (own_ws && cudaMallocAsync(&ws, p.total, st) != cudaSuccess)
+  if (own_ws && cudaMallocAsync(&ws, need, st) != cudaSuccess)
     return cuda_status(cudaErrorMemoryAllocation);
   char *w = static_cast<char *>(ws);
-  float *h = reinterpret_cast<float *>(w + p.off_h);
-  int *sel_idx = reinterpret_cast<int *>(w + p.off_idx);
-  float *sel_sig = reinterpret_cast<float *>(w + p.off_sig);
-  float *a_buf = reinterpret_cast<float *>(w + p.off_a);
-  const int gu_ctas = (int)std::min<int64_t>(dev.num_sms, (int64_t)T * s.d_s);
-
-  cudaError_t e = timed(SFN_STAGE_PRED_H, st,
-                        [&] { return launch_pred_h(s, p.tt_h, x, A, h, B, st); });
-  if (e == cudaSuccess)
-    e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
-      return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, st);
-    });
-  if (e == cudaSuccess)
-    e = timed(SFN_STAGE_GATEUP, st, [&] {
-      return launch_gateup(s, gu_ctas, x, sel_idx, sel_sig, Wg, Wu, Wd, a_buf, dev.err, st);
-    });
-  if (e == cudaSuccess)
-    e = timed(SFN_STAGE_DOWN, st, [&] { return launch_down(s, sel_idx, a_buf, Wd, y, st); });
+  cudaError_t e = cudaSuccess;
+  if (tc) {
+    const TcPlan p = plan_tc(s);
+    uint16_t *h2 = reinterpret_cast<uint16_t *>(w + p.off_h2);
+    float *sig = reinterpret_cast<float *>(w + p.off_sig);
+    uint16_t *act = reinterpret_cast<uint16_t *>(w + p.off_act);
+    uint64_t *m = mask ? mask : reinterpret_cast<uint64_t *>(w + p.off_mask);
+    e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, st); });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
+                [&] { return launch_tc_logits(s, dev, h2, B, nullptr, m, sig, st); });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_TC_GATEUP, st,
+                [&] { return launch_tc_gateup(s, dev, x, Wg, Wu, m, sig, act, st); });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_TC_DOWN, st, [&] { return launch_tc_down(s, dev, act, Wd, y, st); });
+  } else {
+    const GatherPlan p = plan_gather(s);
+    float *h = reinterpret_cast<float *>(w + p.off_h);
+    int *sel_idx = reinterpret_cast<int *>(w + p.off_idx);
+    float *sel_sig = reinterpret_cast<float *>(w + p.off_sig);
+    float *partial = reinterpret_cast<float *>(w + p.off_part);
+    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
+        return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, dev.err, st);
+      });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_FFN, st, [&] {
+        return launch_ffn(s, p.cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, dev.err, st);
+      });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_REDUCE, st,
+                [&] { return launch_reduce_partials(s, p.cpt, partial, y, st); });
+  }
   if (own_ws) {
     cudaError_t ef = cudaFreeAsync(ws, st);
     if (e == cudaSuccess) e = ef;
@@ -307,15 +361,15 @@ size_t sfn_workspace_bytes(int64_t T, int d, int d_i, int r, int bank, int k,
   if (dtype != SFN_DTYPE_BF16 && dtype != SFN_DTYPE_F32) return 0;
   if (check_shape(T, d, d_i, r, bank, k) != SFN_OK || T == 0) return 0;
   if (check_limits(d, d_i, r) != SFN_OK) return 0;
-  return plan_gather(make_shape(T, d, d_i, r, bank, k, dtype == SFN_DTYPE_BF16)).total;
+  return workspace_for(make_shape(T, d, d_i, r, bank, k, dtype == SFN_DTYPE_BF16));
 }
 
 sfn_status sfn_sparse_ffn_forward(const void *x, const void *A, const void *B, const void *Wg,
                                   const void *Wu, const void *Wd, void *y, uint64_t *mask,
                                   int64_t T, int d, int d_i, int r, int bank, int k,
                                   sfn_stream_t stream) {
-  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, nullptr, 0,
-                      true, (cudaStream_t)stream);
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, SFN_PATH_AUTO,
+                      nullptr, 0, true, (cudaStream_t)stream);
 }
 
 sfn_status sfn_sparse_ffn_forward_ws(const void *x, const void *A, const void *B,
@@ -323,16 +377,25 @@ sfn_status sfn_sparse_ffn_forward_ws(const void *x, const void *A, const void *B
                                      uint64_t *mask, int64_t T, int d, int d_i, int r,
                                      int bank, int k, void *workspace, size_t workspace_bytes,
                                      sfn_stream_t stream) {
-  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, workspace,
-                      workspace_bytes, false, (cudaStream_t)stream);
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, SFN_PATH_AUTO,
+                      workspace, workspace_bytes, false, (cudaStream_t)stream);
+}
+
+sfn_status sfn_sparse_ffn_forward_path(const void *x, const void *A, const void *B,
+                                       const void *Wg, const void *Wu, const void *Wd, void *y,
+                                       uint64_t *mask, int64_t T, int d, int d_i, int r,
+                                       int bank, int k, sfn_path path, void *workspace,
+                                       size_t workspace_bytes, sfn_stream_t stream) {
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, path,
+                      workspace, workspace_bytes, false, (cudaStream_t)stream);
 }
 
 sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
                                       const float *Wg, const float *Wu, const float *Wd,
                                       float *y, uint64_t *mask, int64_t T, int d, int d_i,
                                       int r, int bank, int k, sfn_stream_t stream) {
-  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, false, nullptr, 0,
-                      true, (cudaStream_t)stream);
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, false,
+                      SFN_PATH_AUTO, nullptr, 0, true, (cudaStream_t)stream);
 }
 
 sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const float *B,
@@ -340,8 +403,8 @@ sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const f
                                          float *y, uint64_t *mask, int64_t T, int d, int d_i,
                                          int r, int bank, int k, void *workspace,
                                          size_t workspace_bytes, sfn_stream_t stream) {
-  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, false, workspace,
-                      workspace_bytes, false, (cudaStream_t)stream);
+  return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, false,
+                      SFN_PATH_AUTO, workspace, workspace_bytes, false, (cudaStream_t)stream);
 }
 
 sfn_status sfn_timing_begin(void) {
@@ -398,8 +461,12 @@ const char *sfn_stage_name(int stage) {
   switch (stage) {
     case SFN_STAGE_PRED_H: return "pred_h";
     case SFN_STAGE_LOGITS_TOPK: return "logits_topk";
-    case SFN_STAGE_GATEUP: return "gateup";
-    case SFN_STAGE_DOWN: return "down";
+    case SFN_STAGE_FFN: return "ffn";
+    case SFN_STAGE_REDUCE: return "reduce";
+    case SFN_STAGE_TC_H: return "tc_h";
+    case SFN_STAGE_TC_LOGITS_TOPK: return "tc_logits_topk";
+    case SFN_STAGE_TC_GATEUP: return "tc_gateup";
+    case SFN_STAGE_TC_DOWN: return "tc_down";
     case SFN_STAGE_BANK_TOPK: return "bank_topk";
   }
   return "unused";

@@ -6,17 +6,19 @@
 // Training Recipe for Dense-to-Sparse LLMs", gist.science summary,
 // "1. Architectuur" (Executie / Forward Pass) and "3. Hardware Implicaties".
 //
-//   k_gateup_ring  the kept (token, slot) pairs are split evenly over the
-//                  CTAs.  In each CTA one producer thread streams the kept
-//                  W_gate and W_up rows into an 8-stage shared-memory ring
-//                  with 1-D bulk (TMA) copies; 8 consumer warps each own one
-//                  stage and compute g = Wg[j].x, u = Wu[j].x and
-//                  a = sigma(p_j) g u.  The producer also prefetches the
-//                  kept W_down row into L2 for k_down_slices.
-//   k_down_slices  y[t][cols] = sum over the kept slots of a * Wd[j][cols],
-//                  one CTA per (token, 32-column slice), slots summed in a
-//                  fixed order (deterministic), rows read from L2.
-// Only the kept rows of Wg, Wu and Wd are ever read.
+//   k_ffn_ring         one CTA per (token, contiguous range of its kept slots).
+//                      A producer thread streams, for every slot, the kept
+//                      W_gate, W_up and W_down rows into shared-memory rings
+//                      with 1-D bulk (TMA) copies.  S gate/up warps (one per
+//                      ring stage) compute g = Wg[j].x, u = Wu[j].x and
+//                      a = sigma(p_j) g u and hand a to 8 down warps; each
+//                      down warp owns one eighth of the output columns in
+//                      registers and accumulates a * Wd[j, cols] over the
+//                      slots in order.  The CTA writes one fp32 partial row.
+//   k_reduce_partials  y[t] = sum of the token's partial rows in CTA order,
+//                      rounded to the output type.
+// Only the kept rows of Wg, Wu and Wd are read, each once per token; all sums
+// run in a fixed order, so results are bit-reproducible.
 #include "async_util.cuh"
 #include "sfn_internal.cuh"
 
@@ -24,234 +26,272 @@ namespace sfn {
 
 namespace {
 
-constexpr int kMaxStages = 8;          // ring stages = consumer warps (one each)
-constexpr size_t kRingBudget = 200 * 1024;  // shared memory for the ring
-constexpr int kDownThreads = 256;
-constexpr int kSliceCols = 32;
+constexpr int kMaxStages = 8;   // ring stages = gate/up warps (one each)
+constexpr int kDownWarps = 8;   // output column eighths
+constexpr int kMaxChunks = 4;   // 16-byte column chunks per down lane
+constexpr size_t kRingBudget = 192 * 1024;
+constexpr int kMaxSlotsPerCta = 4096;
+constexpr int kReduceThreads = 256;
 
-// blockDim.x = (n_stages + 1) * 32: warps 0..n_stages-1 consume, the last
-// warp produces.
+struct RingLayout {
+  uint32_t row_bytes;
+  int stages;
+  size_t off_gu, off_d, off_a, off_bar, total;
+};
+
+__host__ __device__ inline RingLayout ring_layout(int d, int elt_bytes) {
+  RingLayout L;
+  L.row_bytes = (uint32_t)d * elt_bytes;
+  int s = (int)(kRingBudget / (3ull * L.row_bytes));
+  L.stages = s < 1 ? 1 : (s > kMaxStages ? kMaxStages : s);
+  L.off_gu = 0;
+  L.off_d = L.off_gu + (size_t)L.stages * 2 * L.row_bytes;
+  L.off_a = L.off_d + (size_t)L.stages * L.row_bytes;
+  L.off_bar = L.off_a + (size_t)kMaxSlotsPerCta * sizeof(float);
+  L.total = L.off_bar + 5 * kMaxStages * sizeof(uint64_t);
+  return L;
+}
+
+// blockDim.x = (stages + kDownWarps + 1) * 32: warps [0, S) gate/up,
+// [S, S + 8) down, the last warp produces.  blockIdx.x = t * cpt + c.
 template <class E>
-__global__ void __launch_bounds__((kMaxStages + 1) * 32) k_gateup_ring(
-    const char *__restrict__ x, const int *__restrict__ sel_idx,
-    const float *__restrict__ sel_sig, const char *__restrict__ Wg,
-    const char *__restrict__ Wu, const char *__restrict__ Wd, float *__restrict__ a_out,
-    int64_t n_slots, int d_s, int d, int n_stages, unsigned *err) {
+__global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
+    k_ffn_ring(const char *__restrict__ x, const int *__restrict__ sel_idx,
+               const float *__restrict__ sel_sig, const char *__restrict__ Wg,
+               const char *__restrict__ Wu, const char *__restrict__ Wd,
+               float *__restrict__ partial, int d_s, int d, int cpt, unsigned *err) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const uint32_t row_bytes = (uint32_t)d * E::kBytes;
-  const int kConsumerWarps = n_stages;
-  unsigned char *ring = smem;  // [n_stages][2][row_bytes]
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)n_stages * 2 * row_bytes);
-  uint64_t *empty = full + kMaxStages;
+  const RingLayout L = ring_layout(d, E::kBytes);
+  const int S = L.stages;
+  unsigned char *gu_ring = smem + L.off_gu;  // [S][2][row]
+  unsigned char *d_ring = smem + L.off_d;    // [S][row]
+  float *a_s = reinterpret_cast<float *>(smem + L.off_a);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L.off_bar);
+  uint64_t *gu_full = bar, *gu_empty = bar + kMaxStages, *d_full = bar + 2 * kMaxStages;
+  uint64_t *d_empty = bar + 3 * kMaxStages, *a_ready = bar + 4 * kMaxStages;
 
-  // this CTA's contiguous range of flattened slots f = t * d_s + s
-  const int64_t per = n_slots / gridDim.x, rem = n_slots % gridDim.x;
-  const int64_t f0 = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
-  const int64_t cnt = per + (blockIdx.x < rem ? 1 : 0);
+  const int64_t t = blockIdx.x / cpt;
+  const int c = blockIdx.x % cpt;
+  const int s0 = (int)(((int64_t)d_s * c) / cpt);
+  const int cnt = (int)(((int64_t)d_s * (c + 1)) / cpt) - s0;
+  const int64_t f0 = t * d_s + s0;  // flattened index of the first slot
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kConsumerWarps; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&gu_full[i], 1);
+      mbar_init(&gu_empty[i], 1);
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_empty[i], kDownWarps);
+      mbar_init(&a_ready[i], 1);
     }
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();  // sel_idx and sel_sig come from the previous kernel
   pdl_launch_dependents();
-  pdl_wait();  // sel_idx, sel_sig and x come from earlier work on the stream
 
-  if (warp == kConsumerWarps) {
-    // producer
+  const uint32_t row = L.row_bytes;
+  if (warp == S + kDownWarps) {
+    // ----------------------------------------------------------- producer
     if (lane == 0) {
-      int64_t issued = 0;
-      for (int64_t n = 0; n < cnt; ++n) {
-        const int st = (int)(n % kConsumerWarps);
-        const uint32_t use = (uint32_t)(n / kConsumerWarps);
-        if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1u, err)) break;
+      int issued = 0;
+      for (int n = 0; n < cnt; ++n) {
+        const int st = n % S;
+        const uint32_t use = (uint32_t)(n / S);
+        if (use > 0 && (!mbar_wait(&gu_empty[st], (use - 1) & 1u, err) ||
+                        !mbar_wait(&d_empty[st], (use - 1) & 1u, err)))
+          break;
         const int64_t j = sel_idx[f0 + n];
-        unsigned char *dst = ring + (size_t)st * 2 * row_bytes;
-        mbar_arrive_expect_tx(&full[st], 2 * row_bytes);
-        bulk_g2s(dst, Wg + j * row_bytes, row_bytes, &full[st]);
-        bulk_g2s(dst + row_bytes, Wu + j * row_bytes, row_bytes, &full[st]);
-        prefetch_l2(Wd + j * row_bytes, row_bytes);
+        unsigned char *gdst = gu_ring + (size_t)st * 2 * row;
+        mbar_arrive_expect_tx(&gu_full[st], 2 * row);
+        bulk_g2s(gdst, Wg + j * row, row, &gu_full[st]);
+        bulk_g2s(gdst + row, Wu + j * row, row, &gu_full[st]);
+        mbar_arrive_expect_tx(&d_full[st], row);
+        bulk_g2s(d_ring + (size_t)st * row, Wd + j * row, row, &d_full[st]);
         issued = n + 1;
       }
-      // Do not leave while a copy may still be landing in shared memory:
-      // wait (bounded) for the last issued use of every stage.
-      for (int st = 0; st < kConsumerWarps; ++st) {
-        if (issued <= st) break;
-        const int64_t last = st + ((issued - 1 - st) / kConsumerWarps) * kConsumerWarps;
-        mbar_wait(&full[st], (uint32_t)(last / kConsumerWarps) & 1u, err);
+      // never leave while a copy may still be landing in shared memory
+      for (int st = 0; st < S && st < issued; ++st) {
+        const uint32_t last_use = (uint32_t)((issued - 1 - st) / S);
+        mbar_wait(&gu_full[st], last_use & 1u, err);
+        mbar_wait(&d_full[st], last_use & 1u, err);
       }
     }
     return;
   }
 
-  // consumer warp `warp` owns stage `warp`: slots n = warp, warp + 8, ...
-  const int nchunk = d / E::kVec;
-  const unsigned char *gs = ring + (size_t)warp * 2 * row_bytes;
-  const unsigned char *us = gs + row_bytes;
-  for (int64_t n = warp; n < cnt; n += kConsumerWarps) {
-    if (!mbar_wait(&full[warp], (uint32_t)(n / kConsumerWarps) & 1u, err)) break;
-    const int64_t f = f0 + n;
-    const int64_t t = f / d_s;
+  if (warp < S) {
+    // ----------------------------------------------------------- gate / up
+    const int nchunk = d / E::kVec;
+    const unsigned char *gs = gu_ring + (size_t)warp * 2 * row;
+    const unsigned char *us = gs + row;
     const char *xr = x + t * d * E::kBytes;
-    float g = 0.f, u = 0.f;
+    for (int n = warp; n < cnt; n += S) {
+      if (!mbar_wait(&gu_full[warp], (uint32_t)(n / S) & 1u, err)) break;
+      float g = 0.f, u = 0.f;
 #pragma unroll 4
-    for (int q = lane; q < nchunk; q += 32) {
-      float wg[E::kVec], wu[E::kVec], xv[E::kVec];
-      E::unpack(*reinterpret_cast<const uint4 *>(gs + (size_t)q * 16), wg);
-      E::unpack(*reinterpret_cast<const uint4 *>(us + (size_t)q * 16), wu);
-      E::unpack(ld_nc16(xr + (size_t)q * 16), xv);
+      for (int q = lane; q < nchunk; q += 32) {
+        float wg[E::kVec], wu[E::kVec], xv[E::kVec];
+        E::unpack(*reinterpret_cast<const uint4 *>(gs + (size_t)q * 16), wg);
+        E::unpack(*reinterpret_cast<const uint4 *>(us + (size_t)q * 16), wu);
+        E::unpack(ld_nc16(xr + (size_t)q * 16), xv);
 #pragma unroll
-      for (int e = 0; e < E::kVec; ++e) {
-        g = fmaf(wg[e], xv[e], g);
-        u = fmaf(wu[e], xv[e], u);
+        for (int e = 0; e < E::kVec; ++e) {
+          g = fmaf(wg[e], xv[e], g);
+          u = fmaf(wu[e], xv[e], u);
+        }
+      }
+      g = warp_sum(g);
+      u = warp_sum(u);
+      __syncwarp();
+      if (lane == 0) {
+        a_s[n] = sel_sig[f0 + n] * g * u;
+        mbar_arrive(&gu_empty[warp]);
+        mbar_arrive(&a_ready[warp]);
       }
     }
-    g = warp_sum(g);
-    u = warp_sum(u);
+    return;
+  }
+
+  // ------------------------------------------------------------- down
+  const int dw = warp - S;
+  const int nq = d / E::kVec / kDownWarps;  // 16-byte chunks per down warp
+  float acc[kMaxChunks][E::kVec];
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i)
+#pragma unroll
+    for (int e = 0; e < E::kVec; ++e) acc[i][e] = 0.f;
+  for (int n = 0; n < cnt; ++n) {
+    const int st = n % S;
+    const uint32_t par = (uint32_t)(n / S) & 1u;
+    if (!mbar_wait(&d_full[st], par, err) || !mbar_wait(&a_ready[st], par, err)) break;
+    const float a = a_s[n];
+    const unsigned char *wr = d_ring + (size_t)st * row + (size_t)dw * nq * 16;
+#pragma unroll
+    for (int i = 0; i < kMaxChunks; ++i) {
+      const int q = lane + 32 * i;
+      if (q < nq) {
+        float w[E::kVec];
+        E::unpack(*reinterpret_cast<const uint4 *>(wr + (size_t)q * 16), w);
+#pragma unroll
+        for (int e = 0; e < E::kVec; ++e) acc[i][e] = fmaf(a, w[e], acc[i][e]);
+      }
+    }
     __syncwarp();
-    if (lane == 0) {
-      a_out[f] = sel_sig[f] * g * u;
-      mbar_arrive(&empty[warp]);
+    if (lane == 0) mbar_arrive(&d_empty[st]);
+  }
+  float *out = partial + ((t * cpt) + c) * (int64_t)d + (int64_t)dw * nq * E::kVec;
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int q = lane + 32 * i;
+    if (q < nq) {
+      float4 *dst = reinterpret_cast<float4 *>(out + (size_t)q * E::kVec);
+#pragma unroll
+      for (int e = 0; e < E::kVec / 4; ++e)
+        dst[e] = make_float4(acc[i][4 * e], acc[i][4 * e + 1], acc[i][4 * e + 2], acc[i][4 * e + 3]);
     }
   }
 }
 
-// y[t][c0 .. c0+31] = sum_s a[t][s] * Wd[sel_idx[t][s]][c0 .. c0+31].
-// blockIdx.x = t * n_slices + slice.  A lane reads one 16-byte chunk of one
-// slot's row slice; lanes sharing a chunk index split the slots, and the
-// partial sums are combined in a fixed order (shuffles, then warps in order).
-template <class E>
-__global__ void __launch_bounds__(kDownThreads) k_down_slices(
-    const int *__restrict__ sel_idx, const float *__restrict__ a, const char *__restrict__ Wd,
-    void *__restrict__ y, int d, int d_s, int n_slices) {
-  constexpr int kCpr = kSliceCols / E::kVec;  // 16-byte chunks per slice row
-  constexpr int kRpw = 32 / kCpr;             // slot rows per warp instruction
-  __shared__ float red[kDownThreads / 32][kSliceCols];
-  const int64_t t = blockIdx.x / n_slices;
-  const int c0 = (blockIdx.x % n_slices) * kSliceCols;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane / kCpr, cc = lane % kCpr;
-  const int col = c0 + cc * E::kVec;
-  const bool col_ok = col < d;  // d is a multiple of kVec
-  pdl_launch_dependents();
+// y[t][c0 .. c0+31] = sum_{c < cpt} partial[t][c][c0 .. c0+31].
+// blockIdx.x = t * ceil(d / 32) + slice; thread = (group g = tid / 8, quad q).
+template <bool kBF16>
+__global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
+    const float *__restrict__ partial, void *__restrict__ y, int d, int cpt) {
+  __shared__ float4 red[kReduceThreads / 8][8];
+  const int slices = (d + 31) / 32;
+  const int64_t t = blockIdx.x / slices;
+  const int c0 = (blockIdx.x % slices) * 32;
+  const int g = threadIdx.x >> 3, q = threadIdx.x & 7;
+  const int col = c0 + q * 4;
   pdl_wait();
-
-  const int *idx = sel_idx + t * d_s;
-  const float *av = a + t * d_s;
-  float acc[E::kVec];
-#pragma unroll
-  for (int e = 0; e < E::kVec; ++e) acc[e] = 0.f;
-  constexpr int kStride = (kDownThreads / 32) * kRpw;  // slots per CTA sweep
-  int s = warp * kRpw + sub;
-  // 8 independent row loads in flight per lane per batch
-  for (; s + 7 * kStride < d_s; s += 8 * kStride) {
-    uint4 v[8];
-    float w8[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int64_t j = idx[s + u * kStride];
-      w8[u] = av[s + u * kStride];
-      v[u] = col_ok ? ld_nc16(Wd + (j * d + col) * E::kBytes) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float w[E::kVec];
-      E::unpack(v[u], w);
-#pragma unroll
-      for (int e = 0; e < E::kVec; ++e) acc[e] = fmaf(w8[u], w[e], acc[e]);
+  pdl_launch_dependents();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (col < d) {
+    const float *p = partial + t * cpt * (int64_t)d + col;
+#pragma unroll 4
+    for (int c = g; c < cpt; c += kReduceThreads / 8) {
+      const float4 v = *reinterpret_cast<const float4 *>(p + (int64_t)c * d);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
   }
-  for (; s < d_s; s += kStride) {
-    const int64_t j = idx[s];
-    const float wa = av[s];
-    float w[E::kVec];
-    E::unpack(col_ok ? ld_nc16(Wd + (j * d + col) * E::kBytes) : make_uint4(0, 0, 0, 0), w);
-#pragma unroll
-    for (int e = 0; e < E::kVec; ++e) acc[e] = fmaf(wa, w[e], acc[e]);
-  }
-  // combine lanes with the same chunk index (fixed butterfly order)
-#pragma unroll
-  for (int o = kCpr; o < 32; o <<= 1)
-#pragma unroll
-    for (int e = 0; e < E::kVec; ++e) acc[e] += __shfl_xor_sync(kFull, acc[e], o);
-  if (sub == 0) {
-#pragma unroll
-    for (int e = 0; e < E::kVec; ++e) red[warp][cc * E::kVec + e] = acc[e];
-  }
+  red[g][q] = acc;
   __syncthreads();
-  if (threadIdx.x < kSliceCols) {
-    const int c = c0 + threadIdx.x;
+  if (threadIdx.x < 32) {
+    const int qq = threadIdx.x >> 2, e = threadIdx.x & 3;
     float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDownThreads / 32; ++w) v += red[w][threadIdx.x];
-    if (c < d) {
-      if (E::kBytes == 2)
-        reinterpret_cast<uint16_t *>(y)[t * d + c] = f32_to_bf16_bits(v);
+    for (int gg = 0; gg < kReduceThreads / 8; ++gg) {
+      const float4 r4 = red[gg][qq];
+      v += (e == 0) ? r4.x : (e == 1) ? r4.y : (e == 2) ? r4.z : r4.w;
+    }
+    const int cc = c0 + threadIdx.x;
+    if (cc < d) {
+      if (kBF16)
+        reinterpret_cast<uint16_t *>(y)[t * d + cc] = f32_to_bf16_bits(v);
       else
-        reinterpret_cast<float *>(y)[t * d + c] = v;
+        reinterpret_cast<float *>(y)[t * d + cc] = v;
     }
   }
 }
 
-}  // namespace
-size_t gateup_smem_bytes(const FwdShape &s);
-namespace {
-
-int gateup_stages(const FwdShape &s) {
-  const size_t stage = (size_t)2 * s.d * (s.bf16 ? 2 : 4);
-  int n = (int)(kRingBudget / stage);
-  return n < 1 ? 1 : (n > kMaxStages ? kMaxStages : n);
-}
-
 template <class E>
-cudaError_t gateup_e(const FwdShape &s, int ctas, const void *x, const int *sel_idx,
-                     const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
-                     float *a_out, unsigned *err, cudaStream_t st) {
-  const int n_stages = gateup_stages(s);
-  const size_t smem = gateup_smem_bytes(s);
-  auto kern = k_gateup_ring<E>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
+cudaError_t ffn_e(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
+                  const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
+                  float *partial, unsigned *err, cudaStream_t st) {
+  const RingLayout L = ring_layout(s.d, E::kBytes);
+  auto kern = k_ffn_ring<E>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), L.total);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kern, dim3(ctas), dim3((n_stages + 1) * 32), smem, st, (const char *)x,
-                 sel_idx, sel_sig, (const char *)Wg, (const char *)Wu, (const char *)Wd, a_out,
-                 (int64_t)s.T * s.d_s, s.d_s, s.d, n_stages, err);
-  count_launches(1);
-  return e;
-}
-
-template <class E>
-cudaError_t down_e(const FwdShape &s, const int *sel_idx, const float *a, const void *Wd,
-                   void *y, cudaStream_t st) {
-  const int n_slices = (s.d + kSliceCols - 1) / kSliceCols;
-  const int64_t blocks = (int64_t)n_slices * s.T;
+  const int64_t blocks = (int64_t)cpt * s.T;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e = launch_pdl(k_down_slices<E>, dim3((unsigned)blocks), dim3(kDownThreads), 0,
-                             st, sel_idx, a, (const char *)Wd, y, s.d, s.d_s, n_slices);
+  e = launch_pdl(kern, dim3((unsigned)blocks), dim3((L.stages + kDownWarps + 1) * 32), L.total,
+                 st, (const char *)x, sel_idx, sel_sig, (const char *)Wg, (const char *)Wu,
+                 (const char *)Wd, partial, s.d_s, s.d, cpt, err);
   count_launches(1);
   return e;
 }
 
 }  // namespace
 
-size_t gateup_smem_bytes(const FwdShape &s) {
-  return (size_t)gateup_stages(s) * 2 * s.d * (s.bf16 ? 2 : 4) + 2 * kMaxStages * sizeof(uint64_t);
+bool ffn_shape_ok(const FwdShape &s) {
+  const int elt = s.bf16 ? 2 : 4;
+  const int vec = 16 / elt;
+  return s.d % (vec * kDownWarps) == 0 && s.d / vec / kDownWarps <= 32 * kMaxChunks;
 }
 
-cudaError_t launch_gateup(const FwdShape &s, int ctas, const void *x, const int *sel_idx,
-                          const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
-                          float *a_out, unsigned *err, cudaStream_t st) {
-  if (s.bf16) return gateup_e<EltBF16>(s, ctas, x, sel_idx, sel_sig, Wg, Wu, Wd, a_out, err, st);
-  return gateup_e<EltF32>(s, ctas, x, sel_idx, sel_sig, Wg, Wu, Wd, a_out, err, st);
+int ffn_ctas_per_token(const FwdShape &s, int num_sms) {
+  int64_t cpt = num_sms / s.T;
+  if (cpt < 1) cpt = 1;
+  const int64_t min_cpt = (s.d_s + kMaxSlotsPerCta - 1) / kMaxSlotsPerCta;
+  if (cpt < min_cpt) cpt = min_cpt;
+  if (cpt > s.d_s) cpt = s.d_s;
+  return (int)cpt;
 }
 
-cudaError_t launch_down(const FwdShape &s, const int *sel_idx, const float *a, const void *Wd,
-                        void *y, cudaStream_t st) {
-  if (s.bf16) return down_e<EltBF16>(s, sel_idx, a, Wd, y, st);
-  return down_e<EltF32>(s, sel_idx, a, Wd, y, st);
+cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
+                       const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
+                       float *partial, unsigned *err, cudaStream_t st) {
+  if (s.bf16) return ffn_e<EltBF16>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, err, st);
+  return ffn_e<EltF32>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, err, st);
+}
+
+cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
+                                   cudaStream_t st) {
+  const int64_t blocks = (int64_t)((s.d + 31) / 32) * s.T;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  cudaError_t e;
+  if (s.bf16)
+    e = launch_pdl(k_reduce_partials<true>, dim3((unsigned)blocks), dim3(kReduceThreads), 0, st,
+                   partial, y, s.d, cpt);
+  else
+    e = launch_pdl(k_reduce_partials<false>, dim3((unsigned)blocks), dim3(kReduceThreads), 0, st,
+                   partial, y, s.d, cpt);
+  count_launches(1);
+  return e;
 }
 
 }  // namespace sfn

@@ -7,16 +7,18 @@
 //
 //   k_pred_h       h[t] = A x[t] (fp32), one warp per row of A with the whole
 //                  row's 16-byte loads in flight; token groups of TT share
-//                  each row load.  The first token group also issues L2
-//                  prefetches of B, so that k_logits_topk reads B from L2.
+//                  each row load.
 //   k_logits_topk  p[t] = B h[t] for one bank, then (optionally) that bank's
 //                  top-k: mask word, kept channel ids and sigma(p) in
-//                  ascending channel order (one CTA per bank and token group)
+//                  ascending channel order (one CTA per bank and token group).
+//                  The bank's block of B (64 contiguous rows) is bulk-copied
+//                  into shared memory in the prologue, while k_pred_h runs.
 //   k_bank_topk    standalone top-k on float32 logits (one warp per bank)
 //
-// Both chained kernels use programmatic dependent launch: they let the next
-// kernel start early, issue only L2 prefetches of weights before
-// griddepcontrol.wait, and touch every other buffer after it.
+// The chained kernels use programmatic dependent launch.  Each calls
+// griddepcontrol.wait before touching anything an earlier kernel writes and
+// only then lets its dependent start, so a dependent's prologue (which reads
+// nothing but weights) always runs after all work before its predecessor.
 #include "async_util.cuh"
 #include "sfn_internal.cuh"
 
@@ -26,6 +28,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kThreadsH = 128;          // k_pred_h: 4 rows of A per CTA
+constexpr int kWarpsH = kThreadsH / 32;
+constexpr uint32_t kMaxBBlock = 96 * 1024;  // bank block of B staged in smem
 
 // Stage TT token rows of x (element type E) into shared memory as float;
 // rows past the end of the batch are zero.
@@ -51,31 +56,19 @@ __device__ __forceinline__ void stage_rows(float *xs, const char *x, int64_t t0,
 }
 
 // h[t][m] = sum_n A[m][n] x[t][n].  1-D grid over (token group, row block):
-// blockIdx.x = token_group * ceil(r / kWarps) + row_block.
-// If Bpf != nullptr, the CTAs of token group 0 prefetch B (Bpf_bytes) to L2.
+// blockIdx.x = token_group * ceil(r / kWarpsH) + row_block.
 template <class E, int TT>
-__global__ void __launch_bounds__(kThreads) k_pred_h(const char *__restrict__ x,
-                                                     const char *__restrict__ A,
-                                                     float *__restrict__ h, int64_t T, int d,
-                                                     int r, const char *__restrict__ Bpf,
-                                                     int64_t Bpf_bytes) {
+__global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x,
+                                                      const char *__restrict__ A,
+                                                      float *__restrict__ h, int64_t T, int d,
+                                                      int r) {
   extern __shared__ float4 smem_f4[];
   float *xs = reinterpret_cast<float *>(smem_f4);
-  const int row_blocks = (r + kWarps - 1) / kWarps;
+  const int row_blocks = (r + kWarpsH - 1) / kWarpsH;
   const int64_t tg = blockIdx.x / row_blocks;
   const int rb = blockIdx.x % row_blocks;
-  pdl_launch_dependents();
-  if (Bpf != nullptr && tg == 0 && threadIdx.x == 0) {
-    // this CTA's 16-byte-aligned share of B
-    const int64_t share = ((Bpf_bytes + row_blocks - 1) / row_blocks + 15) / 16 * 16;
-    const int64_t beg = rb * share;
-    const int64_t end = beg + share < Bpf_bytes ? beg + share : Bpf_bytes;
-    for (int64_t o = beg; o < end; o += 65536) {
-      const int64_t n = end - o < 65536 ? end - o : 65536;
-      prefetch_l2(Bpf + o, (uint32_t)n);
-    }
-  }
   pdl_wait();
+  pdl_launch_dependents();
 
   const int64_t t0 = tg * TT;
   const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
@@ -83,7 +76,7 @@ __global__ void __launch_bounds__(kThreads) k_pred_h(const char *__restrict__ x,
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = rb * kWarps + warp;
+  const int m = rb * kWarpsH + warp;
   if (m >= r) return;
   const int nchunk = d / E::kVec;
   const char *row = A + (int64_t)m * d * E::kBytes;
@@ -126,31 +119,58 @@ __global__ void __launch_bounds__(kThreads) k_pred_h(const char *__restrict__ x,
 //   mask    : if non-null, [T][n_banks] uint64
 //   sel_idx : if kTopk, [T][d_s] channel ids of kept channels, bank-major,
 //             ascending inside each bank; sel_sig the matching sigma(p)
-template <class E, int TT, bool kWriteLogits, bool kTopk>
+// kSmemB: the bank's rows of B are staged in shared memory by bulk copies
+// issued before griddepcontrol.wait (they are weights, not outputs of the
+// previous kernel); otherwise they are read from global memory.
+template <class E, int TT, bool kWriteLogits, bool kTopk, bool kSmemB>
 __global__ void __launch_bounds__(kThreads) k_logits_topk(
     const float *__restrict__ h, const char *__restrict__ B, float *__restrict__ logits,
     uint64_t *__restrict__ mask, int *__restrict__ sel_idx, float *__restrict__ sel_sig,
-    int64_t T, int d_i, int r, int bank, int k) {
+    int64_t T, int d_i, int r, int bank, int k, unsigned *err) {
   extern __shared__ float4 smem_f4[];
-  float *hs = reinterpret_cast<float *>(smem_f4);  // [TT][r]
-  float *ps = hs + TT * r;                         // [TT][64]
+  const uint32_t block_bytes = (uint32_t)bank * r * E::kBytes;
+  unsigned char *bs = reinterpret_cast<unsigned char *>(smem_f4);      // [bank][r] (kSmemB)
+  float *hs = reinterpret_cast<float *>(bs + (kSmemB ? block_bytes : 0));  // [TT][r]
+  float *ps = hs + TT * r;                                              // [TT][64]
+  uint64_t *bbar = reinterpret_cast<uint64_t *>(ps + TT * 64);
   const int n_banks = d_i / bank;
   const int b = blockIdx.x % n_banks;
   const int64_t t0 = (int64_t)(blockIdx.x / n_banks) * TT;
   const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
-  pdl_launch_dependents();
+  const char *bblock = B + (int64_t)b * block_bytes;
+  if (kSmemB) {
+    if (threadIdx.x == 0) {
+      mbar_init(bbar, 1);
+      fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(bbar, block_bytes);
+      for (uint32_t o = 0; o < block_bytes; o += 16384) {
+        const uint32_t n = block_bytes - o < 16384 ? block_bytes - o : 16384;
+        bulk_g2s(bs + o, bblock + o, n, bbar);
+      }
+    }
+  }
   pdl_wait();
+  pdl_launch_dependents();
   for (int i = threadIdx.x; i < TT * r; i += blockDim.x) {
     const int t = i / r;
     hs[i] = (t < nt) ? h[(t0 + t) * r + (i - t * r)] : 0.f;
   }
   __syncthreads();
+  bool ok = true;
+  if (kSmemB) {
+    ok = __syncthreads_and(mbar_wait(bbar, 0, err)) != 0;
+    // on a timeout, do not leave while the copies may still land
+    if (!ok && threadIdx.x == 0) mbar_wait(bbar, 0, err);
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunk = r / E::kVec;
   // Each warp owns rows jl = warp + kWarps * i; a group of 4 rows x 2 chunk
   // columns of loads is issued before any arithmetic.
-  for (int jl0 = warp; jl0 < bank; jl0 += 4 * kWarps) {
+  for (int jl0 = warp; ok && jl0 < bank; jl0 += 4 * kWarps) {
     float acc[4][TT];
 #pragma unroll
     for (int q = 0; q < 4; ++q)
@@ -161,12 +181,16 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int jl = jl0 + q * kWarps;
-        const char *row = B + (int64_t)(b * bank + jl) * r * E::kBytes;
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int c = c0 + 32 * u;
-          v[q][u] = (jl < bank && c < nchunk) ? ld_nc16(row + (int64_t)c * 16)
-                                              : make_uint4(0, 0, 0, 0);
+          const bool in = jl < bank && c < nchunk;
+          if (kSmemB)
+            v[q][u] = in ? *reinterpret_cast<const uint4 *>(bs + ((size_t)jl * r + (size_t)c * E::kVec) * E::kBytes)
+                         : make_uint4(0, 0, 0, 0);
+          else
+            v[q][u] = in ? ld_nc16(bblock + ((int64_t)jl * r + (int64_t)c * E::kVec) * E::kBytes)
+                         : make_uint4(0, 0, 0, 0);
         }
       }
 #pragma unroll
@@ -200,7 +224,7 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
       }
     }
   }
-  if (!kTopk) return;
+  if (!kTopk || !ok) return;
   __syncthreads();
 
   const int d_s = n_banks * k;
@@ -241,31 +265,32 @@ __global__ void __launch_bounds__(kThreads) k_bank_topk(const float *__restrict_
 
 template <class E, int TT>
 cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, float *h,
-                      const void *Bpf, cudaStream_t st) {
+                      cudaStream_t st) {
   const size_t smem = (size_t)TT * s.d * sizeof(float);
   auto kern = k_pred_h<E, TT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
-  const int64_t blocks = (int64_t)((s.r + kWarps - 1) / kWarps) * ((s.T + TT - 1) / TT);
+  const int64_t blocks = (int64_t)((s.r + kWarpsH - 1) / kWarpsH) * ((s.T + TT - 1) / TT);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const int64_t bpf_bytes = (int64_t)s.d_i * s.r * (s.bf16 ? 2 : 4);
-  e = launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreads), smem, st, (const char *)x,
-                 (const char *)A, h, s.T, s.d, s.r, (const char *)Bpf, bpf_bytes);
+  e = launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreadsH), smem, st, (const char *)x,
+                 (const char *)A, h, s.T, s.d, s.r);
   count_launches(1);
   return e;
 }
 
-template <class E, int TT, bool W, bool K>
+template <class E, int TT, bool W, bool K, bool SB>
 cudaError_t logits_tt(const FwdShape &s, const float *h, const void *B, float *logits,
-                      uint64_t *mask, int *sel_idx, float *sel_sig, cudaStream_t st) {
-  const size_t smem = (size_t)TT * (s.r + 64) * sizeof(float);
-  auto kern = k_logits_topk<E, TT, W, K>;
+                      uint64_t *mask, int *sel_idx, float *sel_sig, unsigned *err,
+                      cudaStream_t st) {
+  const size_t block = SB ? (size_t)s.bank * s.r * E::kBytes : 0;
+  const size_t smem = block + (size_t)TT * (s.r + 64) * sizeof(float) + 16;
+  auto kern = k_logits_topk<E, TT, W, K, SB>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)s.n_banks * ((s.T + TT - 1) / TT);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   e = launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreads), smem, st, h, (const char *)B,
-                 logits, mask, sel_idx, sel_sig, s.T, s.d_i, s.r, s.bank, s.k);
+                 logits, mask, sel_idx, sel_sig, s.T, s.d_i, s.r, s.bank, s.k, err);
   count_launches(1);
   return e;
 }
@@ -273,52 +298,57 @@ cudaError_t logits_tt(const FwdShape &s, const float *h, const void *B, float *l
 template <class E, bool W, bool K>
 cudaError_t logits_dispatch(const FwdShape &s, int tt, const float *h, const void *B,
                             float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
-                            cudaStream_t st) {
+                            unsigned *err, cudaStream_t st) {
+  const bool sb = (size_t)s.bank * s.r * E::kBytes <= kMaxBBlock;
+#define SFN_LT(TTV)                                                                      \
+  return sb ? logits_tt<E, TTV, W, K, true>(s, h, B, logits, mask, sel_idx, sel_sig, err, st) \
+            : logits_tt<E, TTV, W, K, false>(s, h, B, logits, mask, sel_idx, sel_sig, err, st)
   switch (tt) {
-    case 1: return logits_tt<E, 1, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
-    case 2: return logits_tt<E, 2, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
-    case 4: return logits_tt<E, 4, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
-    default: return logits_tt<E, 8, W, K>(s, h, B, logits, mask, sel_idx, sel_sig, st);
+    case 1: SFN_LT(1);
+    case 2: SFN_LT(2);
+    case 4: SFN_LT(4);
+    default: SFN_LT(8);
   }
+#undef SFN_LT
 }
 
 }  // namespace
 
 cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
-                          const void *Bpf, cudaStream_t st) {
+                          cudaStream_t st) {
   if (s.bf16) {
     switch (tt) {
-      case 1: return pred_h_tt<EltBF16, 1>(s, x, A, h, Bpf, st);
-      case 2: return pred_h_tt<EltBF16, 2>(s, x, A, h, Bpf, st);
-      case 4: return pred_h_tt<EltBF16, 4>(s, x, A, h, Bpf, st);
-      default: return pred_h_tt<EltBF16, 8>(s, x, A, h, Bpf, st);
+      case 1: return pred_h_tt<EltBF16, 1>(s, x, A, h, st);
+      case 2: return pred_h_tt<EltBF16, 2>(s, x, A, h, st);
+      case 4: return pred_h_tt<EltBF16, 4>(s, x, A, h, st);
+      default: return pred_h_tt<EltBF16, 8>(s, x, A, h, st);
     }
   }
   switch (tt) {
-    case 1: return pred_h_tt<EltF32, 1>(s, x, A, h, Bpf, st);
-    case 2: return pred_h_tt<EltF32, 2>(s, x, A, h, Bpf, st);
-    case 4: return pred_h_tt<EltF32, 4>(s, x, A, h, Bpf, st);
-    default: return pred_h_tt<EltF32, 8>(s, x, A, h, Bpf, st);
+    case 1: return pred_h_tt<EltF32, 1>(s, x, A, h, st);
+    case 2: return pred_h_tt<EltF32, 2>(s, x, A, h, st);
+    case 4: return pred_h_tt<EltF32, 4>(s, x, A, h, st);
+    default: return pred_h_tt<EltF32, 8>(s, x, A, h, st);
   }
 }
 
 cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,
                                float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
-                               cudaStream_t st) {
+                               unsigned *err, cudaStream_t st) {
   const bool topk = sel_idx != nullptr;
   const bool write = logits != nullptr;
   if (s.bf16) {
     if (topk && write)
-      return logits_dispatch<EltBF16, true, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+      return logits_dispatch<EltBF16, true, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
     if (topk)
-      return logits_dispatch<EltBF16, false, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
-    return logits_dispatch<EltBF16, true, false>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+      return logits_dispatch<EltBF16, false, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
+    return logits_dispatch<EltBF16, true, false>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
   }
   if (topk && write)
-    return logits_dispatch<EltF32, true, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+    return logits_dispatch<EltF32, true, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
   if (topk)
-    return logits_dispatch<EltF32, false, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
-  return logits_dispatch<EltF32, true, false>(s, tt, h, B, logits, mask, sel_idx, sel_sig, st);
+    return logits_dispatch<EltF32, false, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
+  return logits_dispatch<EltF32, true, false>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
 }
 
 cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,

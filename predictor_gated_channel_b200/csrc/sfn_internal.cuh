@@ -140,7 +140,8 @@ struct FwdShape {
 struct GatherPlan {
   int tt_h;  // tokens per CTA of the h kernel
   int tt_p;  // tokens per CTA of the logits/top-k kernel
-  size_t off_h, off_idx, off_sig, off_a, total;
+  int cpt;   // CTAs per token of the gate/up/down kernel
+  size_t off_h, off_idx, off_sig, off_part, total;
 };
 GatherPlan plan_gather(const FwdShape &s);
 
@@ -165,17 +166,35 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 
 // Launchers (enqueue only; return the launch status).
 cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
-                          const void *Bpf, cudaStream_t st);
+                          cudaStream_t st);
 cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,
                                float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
-                               cudaStream_t st);
+                               unsigned *err, cudaStream_t st);
 cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,
                              int bank, int k, cudaStream_t st);
-size_t gateup_smem_bytes(const FwdShape &s);
-cudaError_t launch_gateup(const FwdShape &s, int ctas, const void *x, const int *sel_idx,
-                          const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
-                          float *a_out, unsigned *err, cudaStream_t st);
-cudaError_t launch_down(const FwdShape &s, const int *sel_idx, const float *a, const void *Wd,
-                        void *y, cudaStream_t st);
+bool ffn_shape_ok(const FwdShape &s);
+int ffn_ctas_per_token(const FwdShape &s, int num_sms);
+cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
+                       const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
+                       float *partial, unsigned *err, cudaStream_t st);
+cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
+                                   cudaStream_t st);
+
+// Scratch carve-up of the tensor-core path.
+struct TcPlan {
+  size_t off_h2, off_sig, off_act, off_mask, total;
+};
+bool tc_shape_ok(const FwdShape &s);
+TcPlan plan_tc(const FwdShape &s);
+cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
+                        uint16_t *h2, cudaStream_t st);
+cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uint16_t *h2,
+                             const void *B, float *logits, uint64_t *mask, float *sig,
+                             cudaStream_t st);
+cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
+                             const void *Wg, const void *Wu, const uint64_t *mask,
+                             const float *sig, uint16_t *act, cudaStream_t st);
+cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
+                           const void *Wd, void *y, cudaStream_t st);
 
 }  // namespace sfn

@@ -1,0 +1,546 @@
+// tc_path.cu -- the many-token path on the 5th-generation tensor cores.
+//
+// The same forward as the few-token path ("Continual LLM Upcycling: A
+// Predictor-Gated Bank-Wise Sparsity Training Recipe for Dense-to-Sparse
+// LLMs", gist.science summary, "1. Architectuur" and "3. Hardware
+// Implicaties"), computed as four tiled contractions over 128-token tiles:
+//
+//   G1  H = X A^T                    -> H split into bf16 hi + lo halves
+//   G2  P = H_hi B^T + H_lo B^T      -> bank top-k fused into the epilogue:
+//                                       mask words + sigma(p) of kept channels
+//                                       (or the raw fp32 logits)
+//   G3  [G | U] = X [W_gate; W_up]^T -> a = sigma(p) g u on kept channels, 0
+//                                       elsewhere (bf16, [T][d_i])
+//   G4  Y = A_act W_down             -> y (bf16)
+//
+// Splitting h = hi + lo keeps the logits fp32-accurate (about 2^-16 relative)
+// although the tensor cores take bf16 operands: B is exactly bf16, so only
+// the error of h - hi - lo (about 2^-17 |h|) remains.
+//
+// Each GEMM is one persistent, warp-specialised kernel (one CTA per SM):
+//   warp 0      TMA producer: tiled loads (128-byte swizzle, no multicast)
+//               into a ring of shared-memory stages
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//               (M 128, N <= 256, K 16, bf16 -> f32) into one of two TMEM
+//               accumulators and commits stage releases / tile completions
+//   warps 2..5  epilogue: tcgen05.ld of the warp's 32 TMEM lanes (= 32 token
+//               rows), the epilogue arithmetic, global stores; they release
+//               the accumulator so the next tile's MMAs overlap this epilogue
+// Every mbarrier wait is bounded (async_util.cuh).
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sfn_internal.cuh"
+#include "tc_util.cuh"
+
+namespace sfn {
+
+namespace {
+
+constexpr int kBM = 128;                       // token rows per tile (UMMA M)
+constexpr int kBK = 64;                        // K per stage: 128-byte rows
+constexpr uint32_t kTileA = kBM * kBK * 2;     // 16 KB
+constexpr int kThreadsTc = 192;
+constexpr int kAccCols = 256;                  // TMEM columns per accumulator
+constexpr size_t kStageBudget = 200 * 1024;
+constexpr int kGroupM = 8;                     // tile rasterisation group
+
+enum : int { kEpiHSplit = 0, kEpiLogits = 1, kEpiTopk = 2, kEpiGateUp = 3, kEpiDown = 4 };
+
+struct TcParams {
+  int64_t T;
+  int tiles_m, tiles_n, k_blocks;
+  int bn;                 // UMMA N
+  int stages;
+  uint32_t stage_bytes;   // bytes delivered per stage (A tiles + B)
+  uint32_t idesc;
+  void *out;              // H2 / logits / a_act / y
+  uint64_t *mask;         // top-k: written; gate/up: read
+  float *sig;             // top-k: written; gate/up: read  ([T][n_banks][k])
+  int ld_out;             // elements per output row
+  int r, k, n_banks;
+  unsigned *err;
+};
+
+template <int kEpi>
+struct EpiTraits {
+  static constexpr int kNumA = (kEpi == kEpiLogits || kEpi == kEpiTopk) ? 2 : 1;
+  static constexpr bool kBMnMajor = (kEpi == kEpiDown);
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &mb,
+                                            int &nb) {
+  const int group = tile / (kGroupM * tiles_n);
+  const int first_m = group * kGroupM;
+  const int gm = min(kGroupM, tiles_m - first_m);
+  const int idx = tile - group * kGroupM * tiles_n;
+  mb = first_m + idx % gm;
+  nb = idx / gm;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  return (uint32_t)f32_to_bf16_bits(a) | ((uint32_t)f32_to_bf16_bits(b) << 16);
+}
+
+// Descending compare-exchange on order keys.
+__device__ __forceinline__ void cex_desc(uint32_t &a, uint32_t &b) {
+  const uint32_t hi = max(a, b), lo = min(a, b);
+  a = hi;
+  b = lo;
+}
+
+// Sort 64 keys in descending order (bitonic network, fully unrolled).
+__device__ __forceinline__ void bitonic_sort64_desc(uint32_t (&s)[64]) {
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          if ((i & size) == 0)
+            cex_desc(s[i], s[j]);
+          else
+            cex_desc(s[j], s[i]);
+        }
+      }
+    }
+  }
+}
+
+template <int kEpi>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    k_tc_gemm(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
+              const __grid_constant__ CUtensorMap tB2, const TcParams p) {
+  using Tr = EpiTraits<kEpi>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)p.stages * p.stage_bytes);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + p.stages;
+  uint64_t *tfull = bars + 2 * p.stages;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *done = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4 * 32);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * kAccCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // operands may come from earlier work on the stream
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tA);
+      prefetch_tmap(&tB);
+      if (kEpi == kEpiGateUp) prefetch_tmap(&tB2);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, p.tiles_m, p.tiles_n, mb, nb);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = (int)(it % p.stages);
+          const uint32_t use = it / p.stages;
+          if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          unsigned char *a = smem + (size_t)s * p.stage_bytes;
+          unsigned char *b = a + Tr::kNumA * kTileA;
+          mbar_arrive_expect_tx(&full[s], p.stage_bytes);
+          tma_load_2d(a, &tA, kb * kBK, mb * kBM, &full[s]);
+          if (Tr::kNumA == 2) tma_load_2d(a + kTileA, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
+          if (kEpi == kEpiGateUp) {
+            tma_load_2d(b, &tB, kb * kBK, nb * 128, &full[s]);
+            tma_load_2d(b + kTileA, &tB2, kb * kBK, nb * 128, &full[s]);
+          } else if (kEpi == kEpiDown) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              tma_load_2d(b + q * 8192, &tB, nb * kAccCols + q * 64, kb * kBK, &full[s]);
+          } else {
+            tma_load_2d(b, &tB, kb * kBK, nb * p.bn, &full[s]);
+          }
+        }
+      }
+      // wait (bounded) until the last load of every stage has landed
+      const uint32_t issued = it;
+      for (int s = 0; s < p.stages && (uint32_t)s < issued; ++s) {
+        const uint32_t last = s + ((issued - 1 - s) / p.stages) * p.stages;
+        mbar_wait(&full[s], (last / p.stages) & 1u, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      uint32_t it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++lt) {
+        const uint32_t acc = lt & 1u, use = lt >> 1;
+        if (use > 0 && !mbar_wait(&tempty[acc], (use - 1) & 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = (int)(it % p.stages);
+          if (!mbar_wait(&full[s], (it / p.stages) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const unsigned char *a = smem + (size_t)s * p.stage_bytes;
+          const unsigned char *b = a + Tr::kNumA * kTileA;
+          const uint64_t adesc = desc_kmajor_sw128(a);
+          const uint64_t adesc2 = desc_kmajor_sw128(a + kTileA);
+          const uint64_t bdesc =
+              Tr::kBMnMajor ? desc_mnmajor_sw128(b, 8192) : desc_kmajor_sw128(b);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t boff = Tr::kBMnMajor ? (uint64_t)(kk * 2048 >> 4) : (uint64_t)(kk * 2);
+            umma_f16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + boff, p.idesc,
+                     (kb > 0 || kk > 0) ? 1u : 0u);
+            if (Tr::kNumA == 2) umma_f16(d_tmem, adesc2 + (uint64_t)(kk * 2), bdesc + boff, p.idesc, 1u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&tfull[acc]);
+      }
+      // all MMAs of this CTA complete before TMEM is released
+      umma_commit(done);
+      mbar_wait(done, 0, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;           // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;    // token row inside the tile
+    uint32_t lt = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
+      int mb, nb;
+      tile_coords(tile, p.tiles_m, p.tiles_n, mb, nb);
+      const uint32_t acc = lt & 1u, use = lt >> 1;
+      if (!mbar_wait(&tfull[acc], use & 1u, p.err)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kAccCols;
+      const int64_t t = (int64_t)mb * kBM + row;
+      const bool valid = t < p.T;
+
+      if (kEpi == kEpiHSplit) {
+        uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
+        for (int c0 = 0; c0 < p.bn; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + c0, v);
+          tmem_ld_wait();
+          if (valid) {
+            const int col = nb * p.bn + c0;
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float f0 = __uint_as_float(v[i]), f1 = __uint_as_float(v[i + 1]);
+              const uint16_t h0 = f32_to_bf16_bits(f0), h1 = f32_to_bf16_bits(f1);
+              const float r0 = f0 - __uint_as_float((uint32_t)h0 << 16);
+              const float r1 = f1 - __uint_as_float((uint32_t)h1 << 16);
+              hi[i / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+              lo[i / 2] = pack_bf16x2(r0, r1);
+            }
+            uint4 *dh = reinterpret_cast<uint4 *>(out + t * p.ld_out + col);
+            uint4 *dl = reinterpret_cast<uint4 *>(out + t * p.ld_out + p.r + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+              dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
+            }
+          }
+        }
+      } else if (kEpi == kEpiLogits || kEpi == kEpiDown) {
+        for (int c0 = 0; c0 < p.bn; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + c0, v);
+          tmem_ld_wait();
+          if (valid) {
+            const int col = nb * p.bn + c0;
+            if (kEpi == kEpiLogits) {
+              uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<float *>(p.out) +
+                                                     t * p.ld_out + col);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) +
+                                                     t * p.ld_out + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                dst[i] = make_uint4(
+                    pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                    pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                    pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                    pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+              }
+            }
+          }
+        }
+      } else if (kEpi == kEpiTopk) {
+        // 4 banks of 64 channels per tile
+        for (int bl = 0; bl < 4; ++bl) {
+          uint32_t v[64];
+          tmem_ld_32x32b_x32(taddr + bl * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld_32x32b_x32(taddr + bl * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          tmem_ld_wait();
+          uint32_t s[64];
+#pragma unroll
+          for (int i = 0; i < 64; ++i) s[i] = order_key(__uint_as_float(v[i]));
+          bitonic_sort64_desc(s);
+          uint32_t tau = s[0];
+#pragma unroll
+          for (int i = 1; i < 64; ++i) tau = (i == p.k - 1) ? s[i] : tau;
+          int gt = 0;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) gt += order_key(__uint_as_float(v[i])) > tau;
+          const int need = p.k - gt;
+          int eq = 0, cnt = 0;
+          uint64_t word = 0;
+          const int bank = nb * 4 + bl;
+          float *sig_out = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const uint32_t key = order_key(__uint_as_float(v[i]));
+            const bool take = key > tau || (key == tau && eq < need);
+            eq += (key == tau);
+            if (take) {
+              word |= 1ull << i;
+              if (valid) sig_out[cnt] = sigmoid_f32(__uint_as_float(v[i]));
+              ++cnt;
+            }
+          }
+          if (valid) p.mask[t * p.n_banks + bank] = word;
+        }
+      } else if (kEpi == kEpiGateUp) {
+        // channels nb*128 .. +127 = banks 2nb, 2nb+1; accumulator columns
+        // 0..127 hold g, 128..255 hold u
+        uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
+        for (int h = 0; h < 2; ++h) {
+          const int bank = nb * 2 + h;
+          const uint64_t word = valid ? p.mask[t * p.n_banks + bank] : 0ull;
+          const float *sig_in = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t g[32], u[32];
+            tmem_ld_32x32b_x32(taddr + h * 64 + c0, g);
+            tmem_ld_32x32b_x32(taddr + 128 + h * 64 + c0, u);
+            tmem_ld_wait();
+            if (valid) {
+              uint32_t packed[16];
+              int rank = __popcll(word & ((1ull << c0) - 1ull));
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                float a2[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const bool on = (word >> (c0 + i + e)) & 1ull;
+                  const float sg = on ? sig_in[rank] : 0.f;
+                  a2[e] = on ? sg * __uint_as_float(g[i + e]) * __uint_as_float(u[i + e]) : 0.f;
+                  rank += on;
+                }
+                packed[i / 2] = pack_bf16x2(a2[0], a2[1]);
+              }
+              uint4 *dst = reinterpret_cast<uint4 *>(out + t * p.ld_out + bank * 64 + c0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
+                                    packed[4 * i + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kAccCols);
+  }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// Row-major bf16 matrix [outer][inner], box {box_inner, box_outer}, 128-byte
+// swizzle, zero fill outside.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int kEpi>
+cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtensorMap &tB2,
+                      TcParams p, int num_sms, cudaStream_t st) {
+  using Tr = EpiTraits<kEpi>;
+  const uint32_t b_bytes = (kEpi == kEpiHSplit) ? (uint32_t)p.bn * 128u : 32768u;
+  p.stage_bytes = Tr::kNumA * kTileA + b_bytes;
+  p.stages = (int)(kStageBudget / p.stage_bytes);
+  if (p.stages > 8) p.stages = 8;
+  p.idesc = idesc_bf16_f32(kBM, p.bn, Tr::kBMnMajor);
+  const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + (2 * p.stages + 5) * 8 + 16;
+  auto kern = k_tc_gemm<kEpi>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const int total = p.tiles_m * p.tiles_n;
+  const int grid = total < num_sms ? total : num_sms;
+  e = launch_pdl(kern, dim3(grid), dim3(kThreadsTc), smem, st, tA, tB, tB2, p);
+  count_launches(1);
+  return e;
+}
+
+}  // namespace
+
+bool tc_shape_ok(const FwdShape &s) {
+  return s.bf16 && s.bank == 64 && s.d % 256 == 0 && s.d_i % 256 == 0 && s.r % 64 == 0 &&
+         s.r <= 512 && s.T > 0 && s.T <= 0x7fffffffLL;
+}
+
+TcPlan plan_tc(const FwdShape &s) {
+  TcPlan p{};
+  size_t off = 0;
+  p.off_h2 = off;
+  off = align_up(off + (size_t)s.T * 2 * s.r * 2, 256);
+  p.off_sig = off;
+  off = align_up(off + (size_t)s.T * s.d_s * 4, 256);
+  p.off_act = off;
+  off = align_up(off + (size_t)s.T * s.d_i * 2, 256);
+  p.off_mask = off;
+  off = align_up(off + (size_t)s.T * s.n_banks * 8, 256);
+  p.total = off;
+  return p;
+}
+
+namespace {
+TcParams base_params(const FwdShape &s, const DeviceInfo &dev) {
+  TcParams p{};
+  p.T = s.T;
+  p.err = dev.err;
+  p.r = s.r;
+  p.k = s.k;
+  p.n_banks = s.n_banks;
+  p.tiles_m = (int)((s.T + kBM - 1) / kBM);
+  return p;
+}
+}  // namespace
+
+// G1: H = X A^T, written as bf16 hi | lo halves of h2 [T][2r].
+cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
+                        uint16_t *h2, cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  const int bn_h = s.r > 256 ? s.r / 2 : s.r;
+  CUtensorMap mX, mA;
+  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mA, A, s.d, s.r, 64, bn_h))
+    return cudaErrorInvalidValue;
+  TcParams p = base_params(s, dev);
+  p.tiles_n = s.r / bn_h;
+  p.k_blocks = s.d / kBK;
+  p.bn = bn_h;
+  p.out = h2;
+  p.ld_out = 2 * s.r;
+  return launch_tc<kEpiHSplit>(mX, mA, mA, p, dev.num_sms, st);
+}
+
+// G2: logits = (H_hi + H_lo) B^T; raw fp32 (logits != nullptr) or the bank
+// top-k fused into the epilogue (mask + sigma(p) of kept channels).
+cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uint16_t *h2,
+                             const void *B, float *logits, uint64_t *mask, float *sig,
+                             cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  CUtensorMap mH, mB;
+  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, kBM) || !make_map(&mB, B, s.r, s.d_i, 64, 256))
+    return cudaErrorInvalidValue;
+  TcParams p = base_params(s, dev);
+  p.tiles_n = s.d_i / 256;
+  p.k_blocks = s.r / kBK;
+  p.bn = 256;
+  if (logits != nullptr) {
+    p.out = logits;
+    p.ld_out = s.d_i;
+    return launch_tc<kEpiLogits>(mH, mB, mB, p, dev.num_sms, st);
+  }
+  p.mask = mask;
+  p.sig = sig;
+  return launch_tc<kEpiTopk>(mH, mB, mB, p, dev.num_sms, st);
+}
+
+// G3: [G | U] = X [Wg; Wu]^T -> act = sigma(p) g u on kept channels, 0 elsewhere.
+cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
+                             const void *Wg, const void *Wu, const uint64_t *mask,
+                             const float *sig, uint16_t *act, cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  CUtensorMap mX, mG, mU;
+  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mG, Wg, s.d, s.d_i, 64, 128) ||
+      !make_map(&mU, Wu, s.d, s.d_i, 64, 128))
+    return cudaErrorInvalidValue;
+  TcParams p = base_params(s, dev);
+  p.tiles_n = s.d_i / 128;
+  p.k_blocks = s.d / kBK;
+  p.bn = 256;
+  p.out = act;
+  p.ld_out = s.d_i;
+  p.mask = const_cast<uint64_t *>(mask);
+  p.sig = const_cast<float *>(sig);
+  return launch_tc<kEpiGateUp>(mX, mG, mU, p, dev.num_sms, st);
+}
+
+// G4: Y = act Wd, with Wd [d_i][d] read as an MN-major B operand.
+cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
+                           const void *Wd, void *y, cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  CUtensorMap mAct, mD;
+  if (!make_map(&mAct, act, s.d_i, s.T, 64, kBM) || !make_map(&mD, Wd, s.d, s.d_i, 64, 64))
+    return cudaErrorInvalidValue;
+  TcParams p = base_params(s, dev);
+  p.tiles_n = s.d / 256;
+  p.k_blocks = s.d_i / kBK;
+  p.bn = 256;
+  p.out = y;
+  p.ld_out = s.d;
+  return launch_tc<kEpiDown>(mAct, mD, mD, p, dev.num_sms, st);
+}
+
+}  // namespace sfn

@@ -99,7 +99,7 @@ def test_workspace_checks(L):
     assert L.sfn_workspace_bytes(-1, 4096, 14336, 448, 64, 16, 0) == 0
     args = [FAKE] * 7 + [None, 1, 4096, 14336, 448, 64, 16]
     assert L.sfn_sparse_ffn_forward_ws(*args, None, need, None) == _capi.SFN_ERR_WORKSPACE
-    assert L.sfn_sparse_ffn_forward_ws(*args, FAKE, need - 1, None) == _capi.SFN_ERR_WORKSPACE
+    assert L.sfn_sparse_ffn_forward_ws(*args, FAKE, 256, None) == _capi.SFN_ERR_WORKSPACE
     assert L.sfn_sparse_ffn_forward_ws(*args, FAKE + 16, need, None) == _capi.SFN_ERR_WORKSPACE
     # scratch grows with T
     assert (L.sfn_workspace_bytes(64, 4096, 14336, 448, 64, 16, 0)

@@ -218,3 +218,64 @@ def test_zero_tokens(full_layer):
     x = torch.empty((0, wl.d), dtype=torch.bfloat16, device=DEV)
     y, mask = _run_forward(dev, x, 64, 16)
     assert y.shape == (0, wl.d) and mask.shape == (0, wl.n_banks)
+
+
+# ------------------------------------------------------------------ tensor path
+
+@pytest.mark.parametrize("T", [1, 5, 128, 130, 300])
+def test_tensor_path_full_width(T, full_layer):
+    """The tcgen05 path (forced) against the oracle, every token checked."""
+    wl, host, dev = full_layer
+    x = make_tokens(WORKLOADS["prefill"], T=T, seed=100 + T)
+    y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
+                                     dev["Wd"], path="tensor")
+    torch.cuda.synchronize()
+    _check_forward(host, x, y, mask, 64, 16, "bf16")
+
+
+@pytest.mark.parametrize("k", [1, 16, 63, 64])
+def test_tensor_path_k_variants(k, full_layer):
+    wl, host, dev = full_layer
+    x = make_tokens(WORKLOADS["prefill"], T=160, seed=200 + k)
+    y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
+                                     dev["Wd"], k=k, path="tensor")
+    torch.cuda.synchronize()
+    rows = np.arange(0, 160, 7)
+    _check_forward(host, x, y, mask, 64, k, "bf16", rows=rows)
+
+
+def test_paths_agree(full_layer):
+    """CUDA-core and tensor paths on the same 96 tokens: masks differ only at
+    allowed near-ties, outputs within the bf16 tolerance of each other."""
+    wl, host, dev = full_layer
+    x = make_tokens(WORKLOADS["prefill"], T=96, seed=7).to(DEV)
+    y1, m1 = sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"],
+                                    path="cuda_core")
+    y2, m2 = sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"],
+                                    path="tensor")
+    torch.cuda.synchronize()
+    same = (m1 == m2).float().mean().item()
+    assert same > 0.99, same
+    rows = torch.nonzero((m1 == m2).all(dim=1)).flatten()
+    err = parity.y_error(y2[rows].float().cpu().numpy(), y1[rows].float().cpu().numpy().astype(np.float64))
+    assert err <= parity.Y_TOL["bf16"], err
+
+
+def test_tensor_predict_logits(full_layer):
+    """sfn_predict at T >= 1024 runs on the tensor cores (split-h logits)."""
+    wl, host, dev = full_layer
+    x = make_tokens(WORKLOADS["prefill"], T=1100, seed=5)
+    got = sfn.predict(x.to(DEV), dev["A"], dev["B"])
+    torch.cuda.synchronize()
+    rows = np.arange(0, 1100, 37)
+    ref = oracle.predict(x[torch.as_tensor(rows)], host["A"], host["B"])
+    err = np.abs(got.cpu().numpy()[rows].astype(np.float64) - ref).max()
+    assert err <= 2e-5 * np.abs(ref).max() + 1e-6, err
+
+
+def test_tensor_path_rejects_unsupported(full_layer):
+    wl, host, dev = full_layer
+    x = make_tokens(wl, T=4).to(DEV)
+    with pytest.raises(sfn.SfnError):
+        sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"],
+                               bank=32, k=8, path="tensor")
