@@ -52,6 +52,8 @@ def parse_args(argv=None):
                     choices=["decode", "batched_decode", "prefill", "long_prefill"])
     ap.add_argument("--impl", default="sfn", choices=["sfn", "reference"])
     ap.add_argument("--k", type=int, default=None, help="override top-k (e.g. 64: dense mask)")
+    ap.add_argument("--path", default="auto", choices=["auto", "cuda_core", "tensor"],
+                    help="kernels to use (the library picks by token count when auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--settle", type=float, default=1.0,
@@ -250,16 +252,19 @@ def run_sfn(args, rank, world, local):
     ms = [torch.empty((T, wl.n_banks), dtype=torch.int64, device=dev) for _ in range(S)]
     ws_bytes = sfn.workspace_bytes(T, wl.d, wl.d_i, wl.r, wl.bank, wl.k, wl.torch_dtype)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    fwd = L.sfn_sparse_ffn_forward_ws if wl.dtype == "bf16" else L.sfn_sparse_ffn_forward_f32_ws
+    path_id = {"auto": 0, "cuda_core": 1, "tensor": 2}[args.path]
     stream = torch.cuda.Stream(device=dev)
 
     def call(i, st_ptr):
         lay = layers[i]
-        rc = fwd(xs[i].data_ptr(), lay["A"].data_ptr(), lay["B"].data_ptr(),
-                 lay["Wg"].data_ptr(), lay["Wu"].data_ptr(), lay["Wd"].data_ptr(),
-                 ys[i].data_ptr(), ms[i].data_ptr(), T, wl.d, wl.d_i, wl.r, wl.bank, wl.k,
-                 ws.data_ptr(), ws_bytes, st_ptr)
-        _capi.check(rc, "sfn_sparse_ffn_forward_ws")
+        ptrs = [xs[i].data_ptr(), lay["A"].data_ptr(), lay["B"].data_ptr(),
+                lay["Wg"].data_ptr(), lay["Wu"].data_ptr(), lay["Wd"].data_ptr(),
+                ys[i].data_ptr(), ms[i].data_ptr(), T, wl.d, wl.d_i, wl.r, wl.bank, wl.k]
+        if wl.dtype == "bf16":
+            rc = L.sfn_sparse_ffn_forward_path(*ptrs, path_id, ws.data_ptr(), ws_bytes, st_ptr)
+        else:
+            rc = L.sfn_sparse_ffn_forward_f32_ws(*ptrs, ws.data_ptr(), ws_bytes, st_ptr)
+        _capi.check(rc, "sfn_sparse_ffn_forward")
 
     # eager warm-up (also compiles kernel attributes outside capture)
     with torch.cuda.stream(stream):
@@ -355,6 +360,8 @@ def run_sfn(args, rank, world, local):
         v["share"] = v["ms_total"] / tot
     work = stage_work(wl, T, union)
     bound = "hbm" if T <= 256 else "tensor"
+    if "tc_down" in stages and "reduce" in stages:  # split-K partial sums
+        work["reduce"] = {"bytes": T * wl.d * 4, "flops": 0}
     dom = max(stages, key=lambda n: stages[n]["ms_total"])
     dom_s = stages[dom]["us_per_launch"] * 1e-6
     if bound == "hbm":
@@ -389,7 +396,7 @@ def run_sfn(args, rank, world, local):
                 lay = layers[i]
                 sfn.sparse_ffn_forward(x_dev, lay["A"], lay["B"], lay["Wg"], lay["Wu"],
                                        lay["Wd"], bank=wl.bank, k=wl.k, y=ys[i], mask=ms[i],
-                                       workspace=ws, stream=stream)
+                                       workspace=ws, path=args.path, stream=stream)
                 y_host.copy_(ys[i], non_blocking=True)
                 m_host.copy_(ms[i], non_blocking=True)
                 stream.synchronize()  # the caller reads the step's result
@@ -430,6 +437,7 @@ def run_sfn(args, rank, world, local):
                    f"({S * sum(v.numel() * v.element_size() for v in layers[0].values()) / 1e9:.2f}"
                    " GB of weights)"),
             "parallelism": f"replica x{world} (token batches independent)",
+            "path": args.path,
             "timing": "CUDA graph replay of the steps, CUDA events on the launching stream",
         },
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,

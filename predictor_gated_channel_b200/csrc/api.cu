@@ -121,11 +121,15 @@ bool device_info(DeviceInfo *out) {
   return true;
 }
 
-GatherPlan plan_gather(const FwdShape &s) {
-  GatherPlan p{};
+int pred_tokens_per_cta(const FwdShape &s) {
   int tt = pow2_tokens(s.T, 8);
   while (tt > 1 && (size_t)tt * s.d * sizeof(float) > kStageBudget) tt /= 2;
-  p.tt_h = tt;
+  return tt;
+}
+
+GatherPlan plan_gather(const FwdShape &s) {
+  GatherPlan p{};
+  p.tt_h = pred_tokens_per_cta(s);
   p.tt_p = pow2_tokens(s.T, 8);
   p.cpt = ffn_ctas_per_token(s, kPlanSms);
   size_t off = 0;
@@ -213,7 +217,7 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
   } else {
     GatherPlan p = plan_gather(s);
     float *h = static_cast<float *>(scratch);
-    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, false, st); });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
         return launch_logits_topk(s, p.tt_p, h, B, logits, nullptr, nullptr, nullptr, dev.err,
@@ -227,6 +231,9 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
 
 // Fewest tokens for which the automatic choice takes the tensor-core path.
 constexpr int64_t kTcMinTokens = 1024;
+// On the tensor path, h = A x runs on CUDA cores up to this many tokens
+// (too few 128-token tiles to spread A over the SMs).
+constexpr int64_t kTcHOnCoresMaxTokens = 256;
 
 bool use_tensor_path(const FwdShape &s, sfn_path path) {
   if (path == SFN_PATH_CUDA_CORE) return false;
@@ -275,22 +282,39 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     float *sig = reinterpret_cast<float *>(w + p.off_sig);
     uint16_t *act = reinterpret_cast<uint16_t *>(w + p.off_act);
     uint64_t *m = mask ? mask : reinterpret_cast<uint64_t *>(w + p.off_mask);
-    e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, st); });
+    // few 128-token tiles: h on CUDA cores (fp32 dot products), written as
+    // the bf16 hi/lo operand of the logits GEMM
+    if (T <= kTcHOnCoresMaxTokens)
+      e = timed(SFN_STAGE_PRED_H, st, [&] {
+        return launch_pred_h(s, pred_tokens_per_cta(s), x, A, h2, true, st);
+      });
+    else
+      e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, st); });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
                 [&] { return launch_tc_logits(s, dev, h2, B, nullptr, m, sig, st); });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_TC_GATEUP, st,
                 [&] { return launch_tc_gateup(s, dev, x, Wg, Wu, m, sig, act, st); });
-    if (e == cudaSuccess)
-      e = timed(SFN_STAGE_TC_DOWN, st, [&] { return launch_tc_down(s, dev, act, Wd, y, st); });
+    if (p.ksplit > 1) {
+      float *part = reinterpret_cast<float *>(w + p.off_part);
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_TC_DOWN, st,
+                  [&] { return launch_tc_down(s, dev, act, Wd, part, p.ksplit, st); });
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_REDUCE, st,
+                  [&] { return launch_reduce_partials(s, p.ksplit, part, y, st); });
+    } else if (e == cudaSuccess) {
+      e = timed(SFN_STAGE_TC_DOWN, st,
+                [&] { return launch_tc_down(s, dev, act, Wd, y, 1, st); });
+    }
   } else {
     const GatherPlan p = plan_gather(s);
     float *h = reinterpret_cast<float *>(w + p.off_h);
     int *sel_idx = reinterpret_cast<int *>(w + p.off_idx);
     float *sel_sig = reinterpret_cast<float *>(w + p.off_sig);
     float *partial = reinterpret_cast<float *>(w + p.off_part);
-    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, st); });
+    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, false, st); });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
         return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, dev.err, st);

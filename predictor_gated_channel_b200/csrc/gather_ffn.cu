@@ -30,13 +30,14 @@ constexpr int kMaxStages = 8;   // ring stages = gate/up warps (one each)
 constexpr int kDownWarps = 8;   // output column eighths
 constexpr int kMaxChunks = 4;   // 16-byte column chunks per down lane
 constexpr size_t kRingBudget = 192 * 1024;
-constexpr int kMaxSlotsPerCta = 4096;
+constexpr int kMaxSlotsPerCta = 1024;
+constexpr uint32_t kMaxXBytes = 16384;  // one token row of x staged in smem
 constexpr int kReduceThreads = 256;
 
 struct RingLayout {
   uint32_t row_bytes;
   int stages;
-  size_t off_gu, off_d, off_a, off_bar, total;
+  size_t off_gu, off_d, off_a, off_idx, off_sig, off_x, off_bar, total;
 };
 
 __host__ __device__ inline RingLayout ring_layout(int d, int elt_bytes) {
@@ -47,7 +48,10 @@ __host__ __device__ inline RingLayout ring_layout(int d, int elt_bytes) {
   L.off_gu = 0;
   L.off_d = L.off_gu + (size_t)L.stages * 2 * L.row_bytes;
   L.off_a = L.off_d + (size_t)L.stages * L.row_bytes;
-  L.off_bar = L.off_a + (size_t)kMaxSlotsPerCta * sizeof(float);
+  L.off_idx = L.off_a + (size_t)kMaxSlotsPerCta * sizeof(float);
+  L.off_sig = L.off_idx + (size_t)kMaxSlotsPerCta * sizeof(int);
+  L.off_x = L.off_sig + (size_t)kMaxSlotsPerCta * sizeof(float);
+  L.off_bar = L.off_x + kMaxXBytes;
   L.total = L.off_bar + 5 * kMaxStages * sizeof(uint64_t);
   return L;
 }
@@ -66,6 +70,9 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
   unsigned char *gu_ring = smem + L.off_gu;  // [S][2][row]
   unsigned char *d_ring = smem + L.off_d;    // [S][row]
   float *a_s = reinterpret_cast<float *>(smem + L.off_a);
+  int *idx_s = reinterpret_cast<int *>(smem + L.off_idx);
+  float *sig_s = reinterpret_cast<float *>(smem + L.off_sig);
+  unsigned char *x_s = smem + L.off_x;
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L.off_bar);
   uint64_t *gu_full = bar, *gu_empty = bar + kMaxStages, *d_full = bar + 2 * kMaxStages;
   uint64_t *d_empty = bar + 3 * kMaxStages, *a_ready = bar + 4 * kMaxStages;
@@ -87,11 +94,18 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
     }
     fence_barrier_init();
   }
-  __syncthreads();
   pdl_wait();  // sel_idx and sel_sig come from the previous kernel
   pdl_launch_dependents();
-
+  // stage this CTA's kept channel ids, their sigma(p) and the token's x
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+    idx_s[i] = sel_idx[f0 + i];
+    sig_s[i] = sel_sig[f0 + i];
+  }
   const uint32_t row = L.row_bytes;
+  for (uint32_t o = threadIdx.x * 16; o < row; o += blockDim.x * 16)
+    *reinterpret_cast<uint4 *>(x_s + o) = ld_nc16(x + t * row + o);
+  __syncthreads();
+
   if (warp == S + kDownWarps) {
     // ----------------------------------------------------------- producer
     if (lane == 0) {
@@ -102,7 +116,7 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
         if (use > 0 && (!mbar_wait(&gu_empty[st], (use - 1) & 1u, err) ||
                         !mbar_wait(&d_empty[st], (use - 1) & 1u, err)))
           break;
-        const int64_t j = sel_idx[f0 + n];
+        const int64_t j = idx_s[n];
         unsigned char *gdst = gu_ring + (size_t)st * 2 * row;
         mbar_arrive_expect_tx(&gu_full[st], 2 * row);
         bulk_g2s(gdst, Wg + j * row, row, &gu_full[st]);
@@ -126,7 +140,6 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
     const int nchunk = d / E::kVec;
     const unsigned char *gs = gu_ring + (size_t)warp * 2 * row;
     const unsigned char *us = gs + row;
-    const char *xr = x + t * d * E::kBytes;
     for (int n = warp; n < cnt; n += S) {
       if (!mbar_wait(&gu_full[warp], (uint32_t)(n / S) & 1u, err)) break;
       float g = 0.f, u = 0.f;
@@ -135,7 +148,7 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
         float wg[E::kVec], wu[E::kVec], xv[E::kVec];
         E::unpack(*reinterpret_cast<const uint4 *>(gs + (size_t)q * 16), wg);
         E::unpack(*reinterpret_cast<const uint4 *>(us + (size_t)q * 16), wu);
-        E::unpack(ld_nc16(xr + (size_t)q * 16), xv);
+        E::unpack(*reinterpret_cast<const uint4 *>(x_s + (size_t)q * 16), xv);
 #pragma unroll
         for (int e = 0; e < E::kVec; ++e) {
           g = fmaf(wg[e], xv[e], g);
@@ -146,7 +159,7 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
       u = warp_sum(u);
       __syncwarp();
       if (lane == 0) {
-        a_s[n] = sel_sig[f0 + n] * g * u;
+        a_s[n] = sig_s[n] * g * u;
         mbar_arrive(&gu_empty[warp]);
         mbar_arrive(&a_ready[warp]);
       }
@@ -260,7 +273,8 @@ cudaError_t ffn_e(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
 bool ffn_shape_ok(const FwdShape &s) {
   const int elt = s.bf16 ? 2 : 4;
   const int vec = 16 / elt;
-  return s.d % (vec * kDownWarps) == 0 && s.d / vec / kDownWarps <= 32 * kMaxChunks;
+  return s.d % (vec * kDownWarps) == 0 && s.d / vec / kDownWarps <= 32 * kMaxChunks &&
+         (uint32_t)s.d * elt <= kMaxXBytes;
 }
 
 int ffn_ctas_per_token(const FwdShape &s, int num_sms) {

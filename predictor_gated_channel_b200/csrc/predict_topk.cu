@@ -57,11 +57,14 @@ __device__ __forceinline__ void stage_rows(float *xs, const char *x, int64_t t0,
 
 // h[t][m] = sum_n A[m][n] x[t][n].  1-D grid over (token group, row block):
 // blockIdx.x = token_group * ceil(r / kWarpsH) + row_block.
-template <class E, int TT>
+// kSplitOut: instead of fp32 h [T][r], write h as two bf16 halves
+// hi = bf16(h), lo = bf16(h - hi) into [T][2r] (hi first), the operand form
+// of the tensor-core logits GEMM.
+template <class E, int TT, bool kSplitOut>
 __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x,
                                                       const char *__restrict__ A,
-                                                      float *__restrict__ h, int64_t T, int d,
-                                                      int r) {
+                                                      void *__restrict__ h_out, int64_t T,
+                                                      int d, int r) {
   extern __shared__ float4 smem_f4[];
   float *xs = reinterpret_cast<float *>(smem_f4);
   const int row_blocks = (r + kWarpsH - 1) / kWarpsH;
@@ -72,24 +75,31 @@ __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x
 
   const int64_t t0 = tg * TT;
   const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
-  stage_rows<E, TT>(xs, x, t0, nt, d);
-  __syncthreads();
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = rb * kWarpsH + warp;
-  if (m >= r) return;
   const int nchunk = d / E::kVec;
-  const char *row = A + (int64_t)m * d * E::kBytes;
+  const char *row = A + (int64_t)(m < r ? m : 0) * d * E::kBytes;
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-  // 16 loads per lane in flight (a whole 8 KB bf16 row per warp)
-  for (int c0 = lane; c0 < nchunk; c0 += 32 * 16) {
-    uint4 v[16];
+  // The row's first 16 loads per lane go out before x is staged, so the
+  // weight fetch overlaps the staging (8 KB bf16 rows: the whole row).
+  uint4 v[16];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int c = c0 + 32 * u;
-      v[u] = (c < nchunk) ? ld_stream16(row + (int64_t)c * 16) : make_uint4(0, 0, 0, 0);
+  for (int u = 0; u < 16; ++u) {
+    const int c = lane + 32 * u;
+    v[u] = (m < r && c < nchunk) ? ld_stream16(row + (int64_t)c * 16) : make_uint4(0, 0, 0, 0);
+  }
+  stage_rows<E, TT>(xs, x, t0, nt, d);
+  __syncthreads();
+  if (m >= r) return;
+  for (int c0 = lane; c0 < nchunk; c0 += 32 * 16) {
+    if (c0 != lane) {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int c = c0 + 32 * u;
+        v[u] = (c < nchunk) ? ld_stream16(row + (int64_t)c * 16) : make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
@@ -109,7 +119,16 @@ __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
     const float v = warp_sum(acc[t]);
-    if (lane == 0 && t < nt) h[(t0 + t) * r + m] = v;
+    if (lane == 0 && t < nt) {
+      if (kSplitOut) {
+        uint16_t *h2 = reinterpret_cast<uint16_t *>(h_out) + (t0 + t) * 2 * r;
+        const uint16_t hi = f32_to_bf16_bits(v);
+        h2[m] = hi;
+        h2[r + m] = f32_to_bf16_bits(v - __uint_as_float((uint32_t)hi << 16));
+      } else {
+        reinterpret_cast<float *>(h_out)[(t0 + t) * r + m] = v;
+      }
+    }
   }
 }
 
@@ -194,19 +213,29 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
         }
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int u = 0; u < 2; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < nchunk) {
+          // this chunk of h, for all tokens, read once and used for 4 rows
+          float hv[TT][E::kVec];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = c0 + 32 * u;
-          if (c < nchunk) {
+          for (int t = 0; t < TT; ++t)
+#pragma unroll
+            for (int e = 0; e < E::kVec; e += 4) {
+              const float4 f = *reinterpret_cast<const float4 *>(hs + t * r + c * E::kVec + e);
+              hv[t][e] = f.x;
+              hv[t][e + 1] = f.y;
+              hv[t][e + 2] = f.z;
+              hv[t][e + 3] = f.w;
+            }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
             float w[E::kVec];
             E::unpack(v[q][u], w);
 #pragma unroll
-            for (int t = 0; t < TT; ++t) {
-              const float *hr = hs + t * r + c * E::kVec;
+            for (int t = 0; t < TT; ++t)
 #pragma unroll
-              for (int e = 0; e < E::kVec; ++e) acc[q][t] = fmaf(w[e], hr[e], acc[q][t]);
-            }
+              for (int e = 0; e < E::kVec; ++e) acc[q][t] = fmaf(w[e], hv[t][e], acc[q][t]);
           }
         }
       }
@@ -263,11 +292,11 @@ __global__ void __launch_bounds__(kThreads) k_bank_topk(const float *__restrict_
   if (lane == 0) mask[wi] = word;
 }
 
-template <class E, int TT>
-cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, float *h,
+template <class E, int TT, bool SPLIT>
+cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, void *h,
                       cudaStream_t st) {
   const size_t smem = (size_t)TT * s.d * sizeof(float);
-  auto kern = k_pred_h<E, TT>;
+  auto kern = k_pred_h<E, TT, SPLIT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)((s.r + kWarpsH - 1) / kWarpsH) * ((s.T + TT - 1) / TT);
@@ -314,22 +343,26 @@ cudaError_t logits_dispatch(const FwdShape &s, int tt, const float *h, const voi
 
 }  // namespace
 
-cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
-                          cudaStream_t st) {
+cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, void *h,
+                          bool split_out, cudaStream_t st) {
+#define SFN_PH(ELT, TTV)                                               \
+  return split_out ? pred_h_tt<ELT, TTV, true>(s, x, A, h, st) \
+                   : pred_h_tt<ELT, TTV, false>(s, x, A, h, st)
   if (s.bf16) {
     switch (tt) {
-      case 1: return pred_h_tt<EltBF16, 1>(s, x, A, h, st);
-      case 2: return pred_h_tt<EltBF16, 2>(s, x, A, h, st);
-      case 4: return pred_h_tt<EltBF16, 4>(s, x, A, h, st);
-      default: return pred_h_tt<EltBF16, 8>(s, x, A, h, st);
+      case 1: SFN_PH(EltBF16, 1);
+      case 2: SFN_PH(EltBF16, 2);
+      case 4: SFN_PH(EltBF16, 4);
+      default: SFN_PH(EltBF16, 8);
     }
   }
   switch (tt) {
-    case 1: return pred_h_tt<EltF32, 1>(s, x, A, h, st);
-    case 2: return pred_h_tt<EltF32, 2>(s, x, A, h, st);
-    case 4: return pred_h_tt<EltF32, 4>(s, x, A, h, st);
-    default: return pred_h_tt<EltF32, 8>(s, x, A, h, st);
+    case 1: SFN_PH(EltF32, 1);
+    case 2: SFN_PH(EltF32, 2);
+    case 4: SFN_PH(EltF32, 4);
+    default: SFN_PH(EltF32, 8);
   }
+#undef SFN_PH
 }
 
 cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,

@@ -144,6 +144,7 @@ struct GatherPlan {
   size_t off_h, off_idx, off_sig, off_part, total;
 };
 GatherPlan plan_gather(const FwdShape &s);
+int pred_tokens_per_cta(const FwdShape &s);
 
 // Launch with programmatic stream serialisation (programmatic dependent
 // launch): the kernel may start while its predecessor in the stream is still
@@ -165,8 +166,8 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // Launchers (enqueue only; return the launch status).
-cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, float *h,
-                          cudaStream_t st);
+cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, void *h,
+                          bool split_out, cudaStream_t st);
 cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,
                                float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
                                unsigned *err, cudaStream_t st);
@@ -182,8 +183,10 @@ cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *part
 
 // Scratch carve-up of the tensor-core path.
 struct TcPlan {
-  size_t off_h2, off_sig, off_act, off_mask, total;
+  int ksplit;  // K ranges of the down GEMM (fp32 partials reduced after)
+  size_t off_h2, off_sig, off_act, off_mask, off_part, total;
 };
+int tc_down_splits(const FwdShape &s, int num_sms);
 bool tc_shape_ok(const FwdShape &s);
 TcPlan plan_tc(const FwdShape &s);
 cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
@@ -195,6 +198,6 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
                              const void *Wg, const void *Wu, const uint64_t *mask,
                              const float *sig, uint16_t *act, cudaStream_t st);
 cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
-                           const void *Wd, void *y, cudaStream_t st);
+                           const void *Wd, void *y, int ksplit, cudaStream_t st);
 
 }  // namespace sfn

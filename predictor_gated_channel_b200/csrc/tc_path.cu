@@ -51,6 +51,7 @@ enum : int { kEpiHSplit = 0, kEpiLogits = 1, kEpiTopk = 2, kEpiGateUp = 3, kEpiD
 struct TcParams {
   int64_t T;
   int tiles_m, tiles_n, k_blocks;
+  int ksplit;             // K ranges per output tile (>1: fp32 partial outputs)
   int bn;                 // UMMA N
   int stages;
   uint32_t stage_bytes;   // bytes delivered per stage (A tiles + B)
@@ -79,6 +80,16 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
   nb = idx / gm;
 }
 
+// Work unit -> output tile and its K-block range [kb0, kb1).
+__device__ __forceinline__ void unit_coords(int unit, const TcParams &p, int &mb, int &nb,
+                                            int &kb0, int &kb1) {
+  const int split = unit % p.ksplit;
+  tile_coords(unit / p.ksplit, p.tiles_m, p.tiles_n, mb, nb);
+  const int per = (p.k_blocks + p.ksplit - 1) / p.ksplit;
+  kb0 = split * per;
+  kb1 = min(p.k_blocks, kb0 + per);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return (uint32_t)f32_to_bf16_bits(a) | ((uint32_t)f32_to_bf16_bits(b) << 16);
 }
@@ -90,23 +101,92 @@ __device__ __forceinline__ void cex_desc(uint32_t &a, uint32_t &b) {
   b = lo;
 }
 
-// Sort 64 keys in descending order (bitonic network, fully unrolled).
-__device__ __forceinline__ void bitonic_sort64_desc(uint32_t (&s)[64]) {
+// Bitonic network sorting s[OFF, OFF + N) in descending order.  Every index
+// is a compile-time constant (the stages are template-recursive), so the
+// array stays in registers.
+template <int OFF, int N, int SIZE, int STRIDE>
+struct BitonicStage {
+  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
 #pragma unroll
-  for (int size = 2; size <= 64; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int j = i ^ stride;
-        if (j > i) {
-          if ((i & size) == 0)
-            cex_desc(s[i], s[j]);
-          else
-            cex_desc(s[j], s[i]);
-        }
+    for (int i = 0; i < N; ++i) {
+      const int j = i ^ STRIDE;
+      if (j > i) {
+        if ((i & SIZE) == 0)
+          cex_desc(s[OFF + i], s[OFF + j]);
+        else
+          cex_desc(s[OFF + j], s[OFF + i]);
       }
     }
+    BitonicStage<OFF, N, SIZE, STRIDE / 2>::run(s);
+  }
+};
+template <int OFF, int N, int SIZE>
+struct BitonicStage<OFF, N, SIZE, 0> {
+  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
+};
+template <int OFF, int N, int SIZE>
+struct BitonicSort {
+  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
+    BitonicStage<OFF, N, SIZE, SIZE / 2>::run(s);
+    BitonicSort<OFF, N, SIZE * 2>::run(s);
+  }
+};
+template <int OFF, int N>
+struct BitonicSort<OFF, N, 2 * N> {
+  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
+};
+
+// s[A..A+16) and s[B..B+16) sorted descending -> s[A..A+16) = the 16 largest
+// of both, sorted descending (max with the reversed other list gives a
+// bitonic sequence, which a half-cleaner cascade sorts).
+template <int A, int B>
+__device__ __forceinline__ void merge_top16(uint32_t (&s)[64]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) s[A + i] = max(s[A + i], s[B + 15 - i]);
+#pragma unroll
+  for (int stride = 8; stride > 0; stride >>= 1)
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if ((i & stride) == 0) cex_desc(s[A + i], s[A + i + stride]);
+}
+
+// Logistic function for the tensor-core epilogues (hardware exp2 based;
+// relative error far below the bf16 rounding of the values it scales).
+__device__ __forceinline__ float sigmoid_fast(float z) {
+  return __frcp_rn(1.0f + __expf(-z));
+}
+
+// k-th largest order key of the 64 logits held in TMEM columns
+// [taddr, taddr + 64) of this thread's row, and the number of keys strictly
+// above it.
+__device__ __forceinline__ void bank_threshold(uint32_t taddr, int k, uint32_t &tau, int &gt) {
+  uint32_t s[64];
+  tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+  tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 64; ++i) s[i] = order_key(__uint_as_float(s[i]));
+  gt = 0;
+  if (k == 16) {
+    BitonicSort<0, 16, 2>::run(s);
+    BitonicSort<16, 16, 2>::run(s);
+    BitonicSort<32, 16, 2>::run(s);
+    BitonicSort<48, 16, 2>::run(s);
+    merge_top16<0, 16>(s);
+    merge_top16<32, 48>(s);
+    // the 16 largest overall: max(s[i], s[47 - i]), i < 16
+    tau = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tau = min(tau, max(s[i], s[47 - i]));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) gt += max(s[i], s[47 - i]) > tau;
+  } else {
+    BitonicSort<0, 64, 2>::run(s);
+    tau = s[0];
+#pragma unroll
+    for (int i = 1; i < 64; ++i) tau = (i == k - 1) ? s[i] : tau;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) gt += s[i] > tau;
   }
 }
 
@@ -127,7 +207,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = p.tiles_m * p.tiles_n;
+  const int total = p.tiles_m * p.tiles_n * p.ksplit;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.stages; ++i) {
@@ -157,10 +237,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (kEpi == kEpiGateUp) prefetch_tmap(&tB2);
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, p.tiles_m, p.tiles_n, mb, nb);
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+      for (int unit = blockIdx.x; unit < total && ok; unit += gridDim.x) {
+        int mb, nb, kb0, kb1;
+        unit_coords(unit, p, mb, nb, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = (int)(it % p.stages);
           const uint32_t use = it / p.stages;
           if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u, p.err)) {
@@ -196,12 +276,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (lane == 0) {
       uint32_t it = 0, lt = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++lt) {
+      for (int unit = blockIdx.x; unit < total && ok; unit += gridDim.x, ++lt) {
+        int mb, nb, kb0, kb1;
+        unit_coords(unit, p, mb, nb, kb0, kb1);
         const uint32_t acc = lt & 1u, use = lt >> 1;
         if (use > 0 && !mbar_wait(&tempty[acc], (use - 1) & 1u, p.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = (int)(it % p.stages);
           if (!mbar_wait(&full[s], (it / p.stages) & 1u, p.err)) {
             ok = false;
@@ -218,7 +300,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t boff = Tr::kBMnMajor ? (uint64_t)(kk * 2048 >> 4) : (uint64_t)(kk * 2);
             umma_f16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + boff, p.idesc,
-                     (kb > 0 || kk > 0) ? 1u : 0u);
+                     (kb > kb0 || kk > 0) ? 1u : 0u);
             if (Tr::kNumA == 2) umma_f16(d_tmem, adesc2 + (uint64_t)(kk * 2), bdesc + boff, p.idesc, 1u);
           }
           umma_commit(&empty[s]);
@@ -234,9 +316,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int q = warp & 3;           // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;    // token row inside the tile
     uint32_t lt = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
-      int mb, nb;
-      tile_coords(tile, p.tiles_m, p.tiles_n, mb, nb);
+    for (int unit = blockIdx.x; unit < total; unit += gridDim.x, ++lt) {
+      int mb, nb, kb0, kb1;
+      unit_coords(unit, p, mb, nb, kb0, kb1);
       const uint32_t acc = lt & 1u, use = lt >> 1;
       if (!mbar_wait(&tfull[acc], use & 1u, p.err)) break;
       tc_fence_after();
@@ -278,9 +360,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           tmem_ld_wait();
           if (valid) {
             const int col = nb * p.bn + c0;
-            if (kEpi == kEpiLogits) {
+            if (kEpi == kEpiLogits || p.ksplit > 1) {
+              // fp32 logits, or fp32 partial sums [T][ksplit][ld_out]
+              const int64_t orow = (p.ksplit > 1) ? t * p.ksplit + unit % p.ksplit : t;
               uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<float *>(p.out) +
-                                                     t * p.ld_out + col);
+                                                     orow * p.ld_out + col);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
                 dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -301,34 +385,29 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       } else if (kEpi == kEpiTopk) {
         // 4 banks of 64 channels per tile
         for (int bl = 0; bl < 4; ++bl) {
-          uint32_t v[64];
-          tmem_ld_32x32b_x32(taddr + bl * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          tmem_ld_32x32b_x32(taddr + bl * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-          tmem_ld_wait();
-          uint32_t s[64];
-#pragma unroll
-          for (int i = 0; i < 64; ++i) s[i] = order_key(__uint_as_float(v[i]));
-          bitonic_sort64_desc(s);
-          uint32_t tau = s[0];
-#pragma unroll
-          for (int i = 1; i < 64; ++i) tau = (i == p.k - 1) ? s[i] : tau;
-          int gt = 0;
-#pragma unroll
-          for (int i = 0; i < 64; ++i) gt += order_key(__uint_as_float(v[i])) > tau;
+          uint32_t tau;
+          int gt;
+          bank_threshold(taddr + bl * 64, p.k, tau, gt);
           const int need = p.k - gt;
           int eq = 0, cnt = 0;
           uint64_t word = 0;
           const int bank = nb * 4 + bl;
           float *sig_out = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const uint32_t key = order_key(__uint_as_float(v[i]));
-            const bool take = key > tau || (key == tau && eq < need);
-            eq += (key == tau);
-            if (take) {
-              word |= 1ull << i;
-              if (valid) sig_out[cnt] = sigmoid_f32(__uint_as_float(v[i]));
-              ++cnt;
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(taddr + bl * 64 + half * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const uint32_t key = order_key(__uint_as_float(v[i]));
+              const bool take = key > tau || (key == tau && eq < need);
+              eq += (key == tau);
+              if (take) {
+                word |= 1ull << (half * 32 + i);
+                if (valid) sig_out[cnt] = sigmoid_fast(__uint_as_float(v[i]));
+                ++cnt;
+              }
             }
           }
           if (valid) p.mask[t * p.n_banks + bank] = word;
@@ -425,7 +504,7 @@ cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtens
   auto kern = k_tc_gemm<kEpi>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
-  const int total = p.tiles_m * p.tiles_n;
+  const int total = p.tiles_m * p.tiles_n * p.ksplit;
   const int grid = total < num_sms ? total : num_sms;
   e = launch_pdl(kern, dim3(grid), dim3(kThreadsTc), smem, st, tA, tB, tB2, p);
   count_launches(1);
@@ -441,6 +520,7 @@ bool tc_shape_ok(const FwdShape &s) {
 
 TcPlan plan_tc(const FwdShape &s) {
   TcPlan p{};
+  p.ksplit = tc_down_splits(s, 148);  // fixed: scratch independent of the device
   size_t off = 0;
   p.off_h2 = off;
   off = align_up(off + (size_t)s.T * 2 * s.r * 2, 256);
@@ -450,6 +530,8 @@ TcPlan plan_tc(const FwdShape &s) {
   off = align_up(off + (size_t)s.T * s.d_i * 2, 256);
   p.off_mask = off;
   off = align_up(off + (size_t)s.T * s.n_banks * 8, 256);
+  p.off_part = off;
+  if (p.ksplit > 1) off = align_up(off + (size_t)s.T * p.ksplit * s.d * 4, 256);
   p.total = off;
   return p;
 }
@@ -463,15 +545,32 @@ TcParams base_params(const FwdShape &s, const DeviceInfo &dev) {
   p.k = s.k;
   p.n_banks = s.n_banks;
   p.tiles_m = (int)((s.T + kBM - 1) / kBM);
+  p.ksplit = 1;
   return p;
 }
 }  // namespace
+
+int tc_down_splits(const FwdShape &s, int num_sms) {
+  const int tiles = (int)((s.T + kBM - 1) / kBM) * (s.d / 256);
+  const int kblocks = s.d_i / kBK;
+  int ks = 1;
+  while (tiles * ks * 2 <= num_sms && ks * 2 <= kblocks / 4) ks *= 2;
+  return ks;
+}
 
 // G1: H = X A^T, written as bf16 hi | lo halves of h2 [T][2r].
 cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
                         uint16_t *h2, cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
-  const int bn_h = s.r > 256 ? s.r / 2 : s.r;
+  // widest tile (r, r/2, else 64 columns) that still gives every SM a tile
+  const int tiles_m = (int)((s.T + kBM - 1) / kBM);
+  int bn_h = 64;
+  for (int cand : {s.r, s.r / 2})
+    if (cand <= 256 && cand % 32 == 0 && s.r % cand == 0 &&
+        (int64_t)tiles_m * (s.r / cand) >= dev.num_sms) {
+      bn_h = cand;
+      break;
+    }
   CUtensorMap mX, mA;
   if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mA, A, s.d, s.r, 64, bn_h))
     return cudaErrorInvalidValue;
@@ -527,9 +626,10 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
   return launch_tc<kEpiGateUp>(mX, mG, mU, p, dev.num_sms, st);
 }
 
-// G4: Y = act Wd, with Wd [d_i][d] read as an MN-major B operand.
+// G4: Y = act Wd, with Wd [d_i][d] read as an MN-major B operand.  With
+// ksplit > 1, y receives fp32 partial sums [T][ksplit][d] instead.
 cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
-                           const void *Wd, void *y, cudaStream_t st) {
+                           const void *Wd, void *y, int ksplit, cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
   CUtensorMap mAct, mD;
   if (!make_map(&mAct, act, s.d_i, s.T, 64, kBM) || !make_map(&mD, Wd, s.d, s.d_i, 64, 64))
@@ -537,6 +637,7 @@ cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint1
   TcParams p = base_params(s, dev);
   p.tiles_n = s.d / 256;
   p.k_blocks = s.d_i / kBK;
+  p.ksplit = ksplit;
   p.bn = 256;
   p.out = y;
   p.ld_out = s.d;

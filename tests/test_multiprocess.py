@@ -1,0 +1,64 @@
+"""Multi-rank host logic of bench.py on CPU (gloo, world size 2).
+
+The path shards by tokens with no collective on the data path; the only
+cross-rank step is the max over ranks of the timed region (the slowest rank
+sets the job's time) and rank 0 alone printing.  These run as two spawned
+processes over gloo on 127.0.0.1.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        assert bench.dist_env() == (rank, world, rank)
+        mx = bench.aggregate_max(10.0 + rank * 5.0, world)
+        # the reference arm runs on rank 0 only; other ranks return at once
+        args = bench.parse_args(["--impl", "reference", "--steps", "1", "--warmup", "1"])
+        ref = bench.run_reference(args, rank, world) if rank != 0 else "skipped"
+        out.put((rank, mx, ref))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_rank0_only_reference():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [15.0, 15.0]
+    assert res[1][2] is None  # rank 1: no reference work, no output
+
+
+def test_value_is_whole_job_aggregate():
+    """value = tokens of all ranks / slowest rank's time (weak scaling)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.aggregate_max(3.0, 1) == 3.0
