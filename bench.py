@@ -156,9 +156,31 @@ def _num(s):
         return None
 
 
+# stage name -> the source files that define its kernel
+KERNEL_SOURCES = {
+    "pred_h": ["predict_topk.cu"], "logits_topk": ["predict_topk.cu"],
+    "predict": ["predict_topk.cu"],
+    "ffn": ["gather_ffn.cu"], "reduce": ["gather_ffn.cu"],
+    "tc_h": ["tc_path.cu", "tc_util.cuh"], "tc_logits_topk": ["tc_path.cu", "tc_util.cuh"],
+    "tc_gateup": ["tc_path.cu", "tc_util.cuh"], "tc_down": ["tc_path.cu", "tc_util.cuh"],
+}
+COMMON_SOURCES = ["sfn_internal.cuh", "async_util.cuh"]
+
+
+def source_digest(kernel):
+    """Digest of the sources a stage's kernel is compiled from."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "predictor_gated_channel_b200", "csrc")
+    for name in sorted(KERNEL_SOURCES.get(kernel, []) + COMMON_SOURCES):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:12]
+
+
 def traffic_from_profiles(kernel, workload):
-    """dram bytes per launch from the committed ncu summary, if it still
-    matches the kernel source (else None)."""
+    """DRAM bytes per launch (read + write) from the committed ncu summary
+    profiles/dram_traffic.txt, if its source digest still matches the
+    kernel's sources; None otherwise."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -166,19 +188,10 @@ def traffic_from_profiles(kernel, workload):
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel \
                 and parts[1] == workload:
-            if parts[3] != source_digest():
+            if parts[3] != source_digest(kernel):
                 return None
             return float(parts[2])
     return None
-
-
-def source_digest():
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "predictor_gated_channel_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
-    return h.hexdigest()[:12]
 
 
 # ------------------------------------------------------------------ algorithmic work
@@ -198,6 +211,8 @@ def stage_work(wl, T, union_channels):
            "flops": 6 * T * d_s * d}
     return {
         "pred_h": pred_h, "logits_topk": logits, "ffn": ffn,
+        "predict": {"bytes": pred_h["bytes"] + logits["bytes"] - T * r * 4,
+                    "flops": pred_h["flops"] + logits["flops"]},
         "reduce": {"bytes": T * d * e, "flops": 0},
         "tc_h": pred_h, "tc_logits_topk": logits,
         "tc_gateup": {"bytes": 2 * union_channels * d * e + T * d * e + T * d_i * e,
@@ -423,7 +438,7 @@ def run_sfn(args, rank, world, local):
 
     value = world * T * K / (elapsed_ms_max * 1e-3)
     # the path's algorithmic minimum: predictor weights, kept rows, x and y
-    step_bytes = sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "ffn", "reduce"))
+    step_bytes = sum(work[n]["bytes"] for n in ("predict", "ffn", "reduce"))
     step_flops = T * useful_flops_per_token(wl)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,

@@ -103,6 +103,10 @@ const char *sfn_status_string(sfn_status s);
 /* ABI version of this header (incremented on any signature change). */
 int sfn_abi_version(void);
 
+/* The CUDA runtime's message for the last SFN_ERR_CUDA returned on this
+ * host thread (static string; "no error" if there was none). */
+const char *sfn_last_error_string(void);
+
 /* Number of kernels this library has launched in this process (all
  * devices, all threads).  Diagnostic counter; never reset. */
 uint64_t sfn_kernel_launch_count(void);
@@ -249,6 +253,7 @@ enum {
   SFN_STAGE_TC_LOGITS_TOPK = 6, /* tensor cores: logits + fused top-k   */
   SFN_STAGE_TC_GATEUP = 7,    /* tensor cores: masked sigma(p) g u      */
   SFN_STAGE_TC_DOWN = 8,      /* tensor cores: y = act W_down           */
+  SFN_STAGE_PREDICT = 9,      /* h, logits and top-k in one cluster kernel */
   SFN_STAGE_COUNT = 16        /* room for the stage ids of this library */
 };
 sfn_status sfn_timing_begin(void);

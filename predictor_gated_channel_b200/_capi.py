@@ -30,6 +30,7 @@ _FWD = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _ci, _ci, _ci, _ci, _ci]
 SIGNATURES = {
     "sfn_status_string": (ctypes.c_char_p, [_ci]),
     "sfn_abi_version": (_ci, []),
+    "sfn_last_error_string": (ctypes.c_char_p, []),
     "sfn_kernel_launch_count": (ctypes.c_uint64, []),
     "sfn_predict": (_ci, [_vp, _vp, _vp, _vp, _i64, _ci, _ci, _ci, _vp]),
     "sfn_predict_f32": (_ci, [_vp, _vp, _vp, _vp, _i64, _ci, _ci, _ci, _vp]),
@@ -56,7 +57,10 @@ _lock = threading.Lock()
 class SfnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)}")
+        msg = f"{where}: {status_string(status)}"
+        if status == SFN_ERR_CUDA:
+            msg += f" ({lib().sfn_last_error_string().decode()})"
+        super().__init__(msg)
 
 
 def lib():

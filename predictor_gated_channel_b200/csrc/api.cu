@@ -183,8 +183,11 @@ FwdShape make_shape(int64_t T, int d, int d_i, int r, int bank, int k, bool bf16
   return s;
 }
 
+thread_local const char *t_last_error = "no error";
+
 sfn_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SFN_OK;
+  t_last_error = cudaGetErrorString(e);
   cudaGetLastError();  // clear a sticky launch error of our own making
   return SFN_ERR_CUDA;
 }
@@ -210,7 +213,8 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
   cudaError_t e;
   if (tc) {
     uint16_t *h2 = static_cast<uint16_t *>(scratch);
-    e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, st); });
+    e = timed(SFN_STAGE_TC_H, st,
+              [&] { return launch_tc_h(s, dev, x, A, h2, nullptr, 1, st); });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
                 [&] { return launch_tc_logits(s, dev, h2, B, logits, nullptr, nullptr, st); });
@@ -231,9 +235,11 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
 
 // Fewest tokens for which the automatic choice takes the tensor-core path.
 constexpr int64_t kTcMinTokens = 1024;
-// On the tensor path, h = A x runs on CUDA cores up to this many tokens
-// (too few 128-token tiles to spread A over the SMs).
-constexpr int64_t kTcHOnCoresMaxTokens = 256;
+// Up to this many tokens the CUDA-core path computes the predictor and the
+// top-k in one cluster kernel (each cluster reads all of A once per token).
+constexpr int64_t kClusterPredictMaxTokens = 2;
+// Devices on which a cluster launch was refused (fall back to two kernels).
+std::atomic<bool> g_cluster_refused[64];
 
 bool use_tensor_path(const FwdShape &s, sfn_path path) {
   if (path == SFN_PATH_CUDA_CORE) return false;
@@ -282,14 +288,20 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     float *sig = reinterpret_cast<float *>(w + p.off_sig);
     uint16_t *act = reinterpret_cast<uint16_t *>(w + p.off_act);
     uint64_t *m = mask ? mask : reinterpret_cast<uint64_t *>(w + p.off_mask);
-    // few 128-token tiles: h on CUDA cores (fp32 dot products), written as
-    // the bf16 hi/lo operand of the logits GEMM
-    if (T <= kTcHOnCoresMaxTokens)
-      e = timed(SFN_STAGE_PRED_H, st, [&] {
-        return launch_pred_h(s, pred_tokens_per_cta(s), x, A, h2, true, st);
-      });
-    else
-      e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, st); });
+    if (p.hsplit > 1) {
+      // few 128-token tiles: split K, then sum the fp32 partials and split
+      // the sum into the bf16 hi/lo operand of the logits GEMM
+      float *hpart = reinterpret_cast<float *>(w + p.off_hpart);
+      e = timed(SFN_STAGE_TC_H, st,
+                [&] { return launch_tc_h(s, dev, x, A, h2, hpart, p.hsplit, st); });
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_REDUCE, st, [&] {
+          return launch_reduce_partials(s, p.hsplit, hpart, h2, st, ReduceOut::kSplitH);
+        });
+    } else {
+      e = timed(SFN_STAGE_TC_H, st,
+                [&] { return launch_tc_h(s, dev, x, A, h2, nullptr, 1, st); });
+    }
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
                 [&] { return launch_tc_logits(s, dev, h2, B, nullptr, m, sig, st); });
@@ -351,6 +363,8 @@ const char *sfn_status_string(sfn_status s) {
 }
 
 int sfn_abi_version(void) { return 1; }
+
+const char *sfn_last_error_string(void) { return t_last_error; }
 
 uint64_t sfn_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -491,6 +505,7 @@ const char *sfn_stage_name(int stage) {
     case SFN_STAGE_TC_LOGITS_TOPK: return "tc_logits_topk";
     case SFN_STAGE_TC_GATEUP: return "tc_gateup";
     case SFN_STAGE_TC_DOWN: return "tc_down";
+    case SFN_STAGE_PREDICT: return "predict";
     case SFN_STAGE_BANK_TOPK: return "bank_topk";
   }
   return "unused";

@@ -7,9 +7,10 @@
 // "1. Architectuur" (Executie / Forward Pass) and "3. Hardware Implicaties".
 //
 //   k_ffn_ring         one CTA per (token, contiguous range of its kept slots).
-//                      A producer thread streams, for every slot, the kept
+//                      A producer warp streams, for every slot, the kept
 //                      W_gate, W_up and W_down rows into shared-memory rings
-//                      with 1-D bulk (TMA) copies.  S gate/up warps (one per
+//                      with 1-D bulk (TMA) copies, one issuing lane per ring
+//                      stage.  S gate/up warps (one per
 //                      ring stage) compute g = Wg[j].x, u = Wu[j].x and
 //                      a = sigma(p_j) g u and hand a to 8 down warps; each
 //                      down warp owns one eighth of the output columns in
@@ -108,10 +109,13 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
 
   if (warp == S + kDownWarps) {
     // ----------------------------------------------------------- producer
-    if (lane == 0) {
+    // Lane st owns ring stage st and issues the copies of slots st, st + S,
+    // ...: several independent issuers keep more row fetches in flight than
+    // one thread issuing every copy in turn.
+    const int st = lane;
+    if (st < S) {
       int issued = 0;
-      for (int n = 0; n < cnt; ++n) {
-        const int st = n % S;
+      for (int n = st; n < cnt; n += S) {
         const uint32_t use = (uint32_t)(n / S);
         if (use > 0 && (!mbar_wait(&gu_empty[st], (use - 1) & 1u, err) ||
                         !mbar_wait(&d_empty[st], (use - 1) & 1u, err)))
@@ -123,13 +127,12 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
         bulk_g2s(gdst + row, Wu + j * row, row, &gu_full[st]);
         mbar_arrive_expect_tx(&d_full[st], row);
         bulk_g2s(d_ring + (size_t)st * row, Wd + j * row, row, &d_full[st]);
-        issued = n + 1;
+        issued = use + 1;
       }
       // never leave while a copy may still be landing in shared memory
-      for (int st = 0; st < S && st < issued; ++st) {
-        const uint32_t last_use = (uint32_t)((issued - 1 - st) / S);
-        mbar_wait(&gu_full[st], last_use & 1u, err);
-        mbar_wait(&d_full[st], last_use & 1u, err);
+      if (issued > 0) {
+        mbar_wait(&gu_full[st], (uint32_t)(issued - 1) & 1u, err);
+        mbar_wait(&d_full[st], (uint32_t)(issued - 1) & 1u, err);
       }
     }
     return;
@@ -207,25 +210,30 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
   }
 }
 
-// y[t][c0 .. c0+31] = sum_{c < cpt} partial[t][c][c0 .. c0+31].
-// blockIdx.x = t * ceil(d / 32) + slice; thread = (group g = tid / 8, quad q).
-template <bool kBF16>
+// out[t][c0 .. c0+C) = sum_{c < cpt} partial[t][c][c0 .. c0+C), summed in a
+// fixed order.  blockIdx.x = t * ceil(n / C) + slice.  Thread = (group g,
+// quad q): group g sums partials c = g, g + G, ...; the G group sums are then
+// added in group order.  kOut: 0 = float32 out, 1 = bf16 out, 2 = bf16 hi/lo
+// halves of h ([T][2n]: hi at column j, lo = bf16(sum - hi) at n + j).
+template <int C, int kOut>
 __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
-    const float *__restrict__ partial, void *__restrict__ y, int d, int cpt) {
-  __shared__ float4 red[kReduceThreads / 8][8];
-  const int slices = (d + 31) / 32;
+    const float *__restrict__ partial, void *__restrict__ out, int n, int cpt) {
+  constexpr int Q = C / 4;                // float4 quads per slice
+  constexpr int G = kReduceThreads / Q;   // partial groups
+  __shared__ float4 red[G][Q];
+  const int slices = (n + C - 1) / C;
   const int64_t t = blockIdx.x / slices;
-  const int c0 = (blockIdx.x % slices) * 32;
-  const int g = threadIdx.x >> 3, q = threadIdx.x & 7;
+  const int c0 = (blockIdx.x % slices) * C;
+  const int g = threadIdx.x / Q, q = threadIdx.x % Q;
   const int col = c0 + q * 4;
   pdl_wait();
   pdl_launch_dependents();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (col < d) {
-    const float *p = partial + t * cpt * (int64_t)d + col;
+  if (col < n) {
+    const float *p = partial + t * cpt * (int64_t)n + col;
 #pragma unroll 4
-    for (int c = g; c < cpt; c += kReduceThreads / 8) {
-      const float4 v = *reinterpret_cast<const float4 *>(p + (int64_t)c * d);
+    for (int c = g; c < cpt; c += G) {
+      const float4 v = *reinterpret_cast<const float4 *>(p + (int64_t)c * n);
       acc.x += v.x;
       acc.y += v.y;
       acc.z += v.z;
@@ -234,19 +242,38 @@ __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
   }
   red[g][q] = acc;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    const int qq = threadIdx.x >> 2, e = threadIdx.x & 3;
-    float v = 0.f;
-    for (int gg = 0; gg < kReduceThreads / 8; ++gg) {
-      const float4 r4 = red[gg][qq];
-      v += (e == 0) ? r4.x : (e == 1) ? r4.y : (e == 2) ? r4.z : r4.w;
+  if (threadIdx.x < Q) {
+    float4 v = red[0][threadIdx.x];
+    for (int gg = 1; gg < G; ++gg) {
+      const float4 r4 = red[gg][threadIdx.x];
+      v.x += r4.x;
+      v.y += r4.y;
+      v.z += r4.z;
+      v.w += r4.w;
     }
-    const int cc = c0 + threadIdx.x;
-    if (cc < d) {
-      if (kBF16)
-        reinterpret_cast<uint16_t *>(y)[t * d + cc] = f32_to_bf16_bits(v);
-      else
-        reinterpret_cast<float *>(y)[t * d + cc] = v;
+    const int cc = c0 + threadIdx.x * 4;
+    if (cc < n) {
+      if (kOut == 0) {
+        *reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + t * n + cc) = v;
+      } else if (kOut == 1) {
+        uint2 o;
+        o.x = (uint32_t)f32_to_bf16_bits(v.x) | ((uint32_t)f32_to_bf16_bits(v.y) << 16);
+        o.y = (uint32_t)f32_to_bf16_bits(v.z) | ((uint32_t)f32_to_bf16_bits(v.w) << 16);
+        *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(out) + t * n + cc) = o;
+      } else {
+        const float f[4] = {v.x, v.y, v.z, v.w};
+        uint16_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = f32_to_bf16_bits(f[e]);
+          lo[e] = f32_to_bf16_bits(f[e] - __uint_as_float((uint32_t)hi[e] << 16));
+        }
+        uint16_t *h2 = reinterpret_cast<uint16_t *>(out) + t * 2 * n;
+        *reinterpret_cast<uint2 *>(h2 + cc) =
+            make_uint2(hi[0] | ((uint32_t)hi[1] << 16), hi[2] | ((uint32_t)hi[3] << 16));
+        *reinterpret_cast<uint2 *>(h2 + n + cc) =
+            make_uint2(lo[0] | ((uint32_t)lo[1] << 16), lo[2] | ((uint32_t)lo[3] << 16));
+      }
     }
   }
 }
@@ -293,17 +320,24 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
   return ffn_e<EltF32>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, err, st);
 }
 
-cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
-                                   cudaStream_t st) {
-  const int64_t blocks = (int64_t)((s.d + 31) / 32) * s.T;
+template <int C>
+cudaError_t reduce_c(const FwdShape &s, int n, int cpt, const float *partial, void *out,
+                     ReduceOut kind, cudaStream_t st) {
+  const int64_t blocks = (int64_t)((n + C - 1) / C) * s.T;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e;
-  if (s.bf16)
-    e = launch_pdl(k_reduce_partials<true>, dim3((unsigned)blocks), dim3(kReduceThreads), 0, st,
-                   partial, y, s.d, cpt);
-  else
-    e = launch_pdl(k_reduce_partials<false>, dim3((unsigned)blocks), dim3(kReduceThreads), 0, st,
-                   partial, y, s.d, cpt);
+  const dim3 grid((unsigned)blocks), block(kReduceThreads);
+  if (kind == ReduceOut::kSplitH)
+    return launch_pdl(k_reduce_partials<C, 2>, grid, block, 0, st, partial, out, n, cpt);
+  if (s.bf16) return launch_pdl(k_reduce_partials<C, 1>, grid, block, 0, st, partial, out, n, cpt);
+  return launch_pdl(k_reduce_partials<C, 0>, grid, block, 0, st, partial, out, n, cpt);
+}
+
+cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
+                                   cudaStream_t st, ReduceOut kind) {
+  const int n = (kind == ReduceOut::kSplitH) ? s.r : s.d;
+  // many partials: narrow slices and 32 partial groups; few: wide slices
+  cudaError_t e = cpt >= 32 ? reduce_c<32>(s, n, cpt, partial, y, kind, st)
+                            : reduce_c<128>(s, n, cpt, partial, y, kind, st);
   count_launches(1);
   return e;
 }

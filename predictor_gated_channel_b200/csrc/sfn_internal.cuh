@@ -173,24 +173,34 @@ cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const 
                                unsigned *err, cudaStream_t st);
 cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,
                              int bank, int k, cudaStream_t st);
+// Cluster size for the fused predictor + top-k kernel (0: not applicable).
+int predict_cluster_size(const FwdShape &s);
+cudaError_t launch_predict_cluster(const FwdShape &s, int cl, const void *x, const void *A,
+                                   const void *B, uint64_t *mask, int *sel_idx,
+                                   float *sel_sig, unsigned *err, cudaStream_t st);
 bool ffn_shape_ok(const FwdShape &s);
 int ffn_ctas_per_token(const FwdShape &s, int num_sms);
 cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
                        const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
                        float *partial, unsigned *err, cudaStream_t st);
+// Output of k_reduce_partials: y in the call's element type, or the bf16
+// hi/lo halves of h ([T][2r], "split").
+enum class ReduceOut { kY, kSplitH };
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
-                                   cudaStream_t st);
+                                   cudaStream_t st, ReduceOut kind = ReduceOut::kY);
 
 // Scratch carve-up of the tensor-core path.
 struct TcPlan {
   int ksplit;  // K ranges of the down GEMM (fp32 partials reduced after)
-  size_t off_h2, off_sig, off_act, off_mask, off_part, total;
+  int hsplit;  // K ranges of the h GEMM (fp32 partials reduced + split after)
+  size_t off_h2, off_sig, off_act, off_mask, off_part, off_hpart, total;
 };
 int tc_down_splits(const FwdShape &s, int num_sms);
+int tc_h_splits(const FwdShape &s, int num_sms);
 bool tc_shape_ok(const FwdShape &s);
 TcPlan plan_tc(const FwdShape &s);
 cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
-                        uint16_t *h2, cudaStream_t st);
+                        uint16_t *h2, float *partial, int ksplit, cudaStream_t st);
 cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uint16_t *h2,
                              const void *B, float *logits, uint64_t *mask, float *sig,
                              cudaStream_t st);

@@ -29,6 +29,7 @@
 // Every mbarrier wait is bounded (async_util.cuh).
 #include <cudaTypedefs.h>
 
+#include <initializer_list>
 #include <mutex>
 
 #include "sfn_internal.cuh"
@@ -43,7 +44,7 @@ constexpr int kBK = 64;                        // K per stage: 128-byte rows
 constexpr uint32_t kTileA = kBM * kBK * 2;     // 16 KB
 constexpr int kThreadsTc = 192;
 constexpr int kAccCols = 256;                  // TMEM columns per accumulator
-constexpr size_t kStageBudget = 200 * 1024;
+constexpr size_t kMaxDynSmem = 232448;            // 227 KB per CTA on sm_100
 constexpr int kGroupM = 8;                     // tile rasterisation group
 
 enum : int { kEpiHSplit = 0, kEpiLogits = 1, kEpiTopk = 2, kEpiGateUp = 3, kEpiDown = 4 };
@@ -150,11 +151,14 @@ __device__ __forceinline__ void merge_top16(uint32_t (&s)[64]) {
       if ((i & stride) == 0) cex_desc(s[A + i], s[A + i + stride]);
 }
 
-// Logistic function for the tensor-core epilogues (hardware exp2 based;
-// relative error far below the bf16 rounding of the values it scales).
+// Logistic function for the tensor-core epilogues (hardware exp2 and
+// reciprocal; relative error far below the bf16 rounding of the values it
+// scales).  Saturates to exactly 0 and 1.
 __device__ __forceinline__ float sigmoid_fast(float z) {
-  return __frcp_rn(1.0f + __expf(-z));
+  return __fdividef(1.0f, 1.0f + __expf(-z));
 }
+
+constexpr int kStageRow = 65;  // floats per epilogue thread row (k <= 64, padded)
 
 // k-th largest order key of the 64 logits held in TMEM columns
 // [taddr, taddr + 64) of this thread's row, and the number of keys strictly
@@ -205,6 +209,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   uint64_t *tempty = tfull + 2;
   uint64_t *done = tempty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  // epilogue staging rows (top-k: kept logits of one bank per thread row)
+  float *stage_rows_smem = reinterpret_cast<float *>(smem + (size_t)p.stages * p.stage_bytes + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = p.tiles_m * p.tiles_n * p.ksplit;
@@ -253,8 +259,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           tma_load_2d(a, &tA, kb * kBK, mb * kBM, &full[s]);
           if (Tr::kNumA == 2) tma_load_2d(a + kTileA, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
           if (kEpi == kEpiGateUp) {
-            tma_load_2d(b, &tB, kb * kBK, nb * 128, &full[s]);
-            tma_load_2d(b + kTileA, &tB2, kb * kBK, nb * 128, &full[s]);
+            tma_load_2d(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
+            tma_load_2d(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
           } else if (kEpi == kEpiDown) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -326,7 +332,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const int64_t t = (int64_t)mb * kBM + row;
       const bool valid = t < p.T;
 
-      if (kEpi == kEpiHSplit) {
+      if (kEpi == kEpiHSplit && p.ksplit == 1) {
         uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
         for (int c0 = 0; c0 < p.bn; c0 += 32) {
           uint32_t v[32];
@@ -353,14 +359,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             }
           }
         }
-      } else if (kEpi == kEpiLogits || kEpi == kEpiDown) {
+      } else if (kEpi == kEpiLogits || kEpi == kEpiDown || kEpi == kEpiHSplit) {
         for (int c0 = 0; c0 < p.bn; c0 += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + c0, v);
           tmem_ld_wait();
           if (valid) {
             const int col = nb * p.bn + c0;
-            if (kEpi == kEpiLogits || p.ksplit > 1) {
+            if (kEpi != kEpiDown || p.ksplit > 1) {
               // fp32 logits, or fp32 partial sums [T][ksplit][ld_out]
               const int64_t orow = (p.ksplit > 1) ? t * p.ksplit + unit % p.ksplit : t;
               uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<float *>(p.out) +
@@ -383,47 +389,62 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
         }
       } else if (kEpi == kEpiTopk) {
-        // 4 banks of 64 channels per tile
-        for (int bl = 0; bl < 4; ++bl) {
+        // bn/64 banks of 64 channels per tile.  The mask pass is branch-free: the
+        // logits of kept channels are compacted, in channel order, into this
+        // thread's staging row; sigma is then evaluated for those k only.
+        float *stg = stage_rows_smem + row * kStageRow;
+        const int banks_per_tile = p.bn / 64;
+        for (int bl = 0; bl < banks_per_tile; ++bl) {
           uint32_t tau;
           int gt;
           bank_threshold(taddr + bl * 64, p.k, tau, gt);
           const int need = p.k - gt;
           int eq = 0, cnt = 0;
-          uint64_t word = 0;
-          const int bank = nb * 4 + bl;
-          float *sig_out = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
+          uint32_t bits[2];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(taddr + bl * 64 + half * 32, v);
             tmem_ld_wait();
+            uint32_t b = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const uint32_t key = order_key(__uint_as_float(v[i]));
-              const bool take = key > tau || (key == tau && eq < need);
+              const bool take = (key > tau) | ((key == tau) & (eq < need));
               eq += (key == tau);
-              if (take) {
-                word |= 1ull << (half * 32 + i);
-                if (valid) sig_out[cnt] = sigmoid_fast(__uint_as_float(v[i]));
-                ++cnt;
-              }
+              b |= (uint32_t)take << i;
+              if (take) stg[cnt] = __uint_as_float(v[i]);
+              cnt += take;
+            }
+            bits[half] = b;
+          }
+          const int bank = nb * banks_per_tile + bl;
+          if (valid) {
+            p.mask[t * p.n_banks + bank] = ((uint64_t)bits[1] << 32) | bits[0];
+            float *sig_out = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
+            if ((p.k & 3) == 0) {
+              for (int s4 = 0; s4 < p.k; s4 += 4)
+                *reinterpret_cast<float4 *>(sig_out + s4) =
+                    make_float4(sigmoid_fast(stg[s4]), sigmoid_fast(stg[s4 + 1]),
+                                sigmoid_fast(stg[s4 + 2]), sigmoid_fast(stg[s4 + 3]));
+            } else {
+              for (int s1 = 0; s1 < p.k; ++s1) sig_out[s1] = sigmoid_fast(stg[s1]);
             }
           }
-          if (valid) p.mask[t * p.n_banks + bank] = word;
         }
       } else if (kEpi == kEpiGateUp) {
-        // channels nb*128 .. +127 = banks 2nb, 2nb+1; accumulator columns
-        // 0..127 hold g, 128..255 hold u
+        // channels nb*bn/2 .. +bn/2-1 (bn/128 banks); accumulator columns
+        // [0, bn/2) hold g, [bn/2, bn) hold u
         uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
-        for (int h = 0; h < 2; ++h) {
-          const int bank = nb * 2 + h;
+        const int half_n = p.bn / 2;
+        for (int h = 0; h < half_n / 64; ++h) {
+          const int bank = nb * (half_n / 64) + h;
           const uint64_t word = valid ? p.mask[t * p.n_banks + bank] : 0ull;
           const float *sig_in = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
           for (int c0 = 0; c0 < 64; c0 += 32) {
             uint32_t g[32], u[32];
             tmem_ld_32x32b_x32(taddr + h * 64 + c0, g);
-            tmem_ld_32x32b_x32(taddr + 128 + h * 64 + c0, u);
+            tmem_ld_32x32b_x32(taddr + half_n + h * 64 + c0, u);
             tmem_ld_wait();
             if (valid) {
               uint32_t packed[16];
@@ -495,12 +516,17 @@ template <int kEpi>
 cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtensorMap &tB2,
                       TcParams p, int num_sms, cudaStream_t st) {
   using Tr = EpiTraits<kEpi>;
-  const uint32_t b_bytes = (kEpi == kEpiHSplit) ? (uint32_t)p.bn * 128u : 32768u;
+  const uint32_t b_bytes = (kEpi == kEpiDown) ? 32768u : (uint32_t)p.bn * 128u;
   p.stage_bytes = Tr::kNumA * kTileA + b_bytes;
-  p.stages = (int)(kStageBudget / p.stage_bytes);
+  const size_t epi_bytes = (kEpi == kEpiTopk) ? (size_t)kBM * kStageRow * sizeof(float) : 0;
+  // as many stages as fit beside the alignment slack, barriers and staging
+  const size_t fixed = 1024 + 256 + epi_bytes;
+  p.stages = (int)(((size_t)kMaxDynSmem - fixed) / p.stage_bytes);
   if (p.stages > 8) p.stages = 8;
+  if (p.stages < 2) return cudaErrorInvalidValue;
   p.idesc = idesc_bf16_f32(kBM, p.bn, Tr::kBMnMajor);
-  const size_t smem = 1024 + (size_t)p.stages * p.stage_bytes + (2 * p.stages + 5) * 8 + 16;
+  const size_t smem = fixed + (size_t)p.stages * p.stage_bytes;
+  if ((2 * p.stages + 5) * 8 + 4 > 256) return cudaErrorInvalidValue;
   auto kern = k_tc_gemm<kEpi>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -521,6 +547,7 @@ bool tc_shape_ok(const FwdShape &s) {
 TcPlan plan_tc(const FwdShape &s) {
   TcPlan p{};
   p.ksplit = tc_down_splits(s, 148);  // fixed: scratch independent of the device
+  p.hsplit = tc_h_splits(s, 148);
   size_t off = 0;
   p.off_h2 = off;
   off = align_up(off + (size_t)s.T * 2 * s.r * 2, 256);
@@ -532,6 +559,8 @@ TcPlan plan_tc(const FwdShape &s) {
   off = align_up(off + (size_t)s.T * s.n_banks * 8, 256);
   p.off_part = off;
   if (p.ksplit > 1) off = align_up(off + (size_t)s.T * p.ksplit * s.d * 4, 256);
+  p.off_hpart = off;
+  if (p.hsplit > 1) off = align_up(off + (size_t)s.T * p.hsplit * s.r * 4, 256);
   p.total = off;
   return p;
 }
@@ -558,28 +587,49 @@ int tc_down_splits(const FwdShape &s, int num_sms) {
   return ks;
 }
 
-// G1: H = X A^T, written as bf16 hi | lo halves of h2 [T][2r].
+// Widest N tile from `cands` (descending) that still gives every SM a tile.
+static int pick_bn(int tiles_m, int n_total, std::initializer_list<int> cands, int num_sms) {
+  int last = 0;
+  for (int c : cands) {
+    if (n_total % c) continue;
+    last = c;
+    if ((int64_t)tiles_m * (n_total / c) >= num_sms) return c;
+  }
+  return last;
+}
+
+int tc_h_splits(const FwdShape &s, int num_sms) {
+  const int tiles = (int)((s.T + kBM - 1) / kBM) * (s.r / 64);
+  const int kblocks = s.d / kBK;
+  int ks = 1;
+  while (tiles * ks * 2 <= num_sms && ks * 2 <= kblocks / 2) ks *= 2;
+  return ks;
+}
+
+// G1: H = X A^T.  ksplit == 1: written as bf16 hi | lo halves of h2 [T][2r];
+// ksplit > 1: fp32 partial sums [T][ksplit][r] into `partial` (the caller
+// reduces them and splits hi/lo).
 cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
-                        uint16_t *h2, cudaStream_t st) {
+                        uint16_t *h2, float *partial, int ksplit, cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
-  // widest tile (r, r/2, else 64 columns) that still gives every SM a tile
   const int tiles_m = (int)((s.T + kBM - 1) / kBM);
-  int bn_h = 64;
-  for (int cand : {s.r, s.r / 2})
-    if (cand <= 256 && cand % 32 == 0 && s.r % cand == 0 &&
-        (int64_t)tiles_m * (s.r / cand) >= dev.num_sms) {
-      bn_h = cand;
-      break;
-    }
+  const int bn_h = ksplit > 1 ? 64
+                              : pick_bn(tiles_m, s.r, {s.r <= 256 ? s.r : s.r / 2, 64}, dev.num_sms);
   CUtensorMap mX, mA;
   if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mA, A, s.d, s.r, 64, bn_h))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
   p.tiles_n = s.r / bn_h;
   p.k_blocks = s.d / kBK;
+  p.ksplit = ksplit;
   p.bn = bn_h;
-  p.out = h2;
-  p.ld_out = 2 * s.r;
+  if (ksplit > 1) {
+    p.out = partial;
+    p.ld_out = s.r;
+  } else {
+    p.out = h2;
+    p.ld_out = 2 * s.r;
+  }
   return launch_tc<kEpiHSplit>(mX, mA, mA, p, dev.num_sms, st);
 }
 
@@ -589,13 +639,15 @@ cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uin
                              const void *B, float *logits, uint64_t *mask, float *sig,
                              cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
+  const int tiles_m = (int)((s.T + kBM - 1) / kBM);
+  const int bn = pick_bn(tiles_m, s.d_i, {256, 128, 64}, dev.num_sms);
   CUtensorMap mH, mB;
-  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, kBM) || !make_map(&mB, B, s.r, s.d_i, 64, 256))
+  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, kBM) || !make_map(&mB, B, s.r, s.d_i, 64, bn))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
-  p.tiles_n = s.d_i / 256;
+  p.tiles_n = s.d_i / bn;
   p.k_blocks = s.r / kBK;
-  p.bn = 256;
+  p.bn = bn;
   if (logits != nullptr) {
     p.out = logits;
     p.ld_out = s.d_i;
@@ -611,14 +663,17 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
                              const void *Wg, const void *Wu, const uint64_t *mask,
                              const float *sig, uint16_t *act, cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
+  const int tiles_m = (int)((s.T + kBM - 1) / kBM);
+  // N tile: g and u of 128 channels (two banks) or of 64 channels (one bank)
+  const int bn = 2 * pick_bn(tiles_m, s.d_i, {128, 64}, dev.num_sms);
   CUtensorMap mX, mG, mU;
-  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mG, Wg, s.d, s.d_i, 64, 128) ||
-      !make_map(&mU, Wu, s.d, s.d_i, 64, 128))
+  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mG, Wg, s.d, s.d_i, 64, bn / 2) ||
+      !make_map(&mU, Wu, s.d, s.d_i, 64, bn / 2))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
-  p.tiles_n = s.d_i / 128;
+  p.tiles_n = s.d_i / (bn / 2);
   p.k_blocks = s.d / kBK;
-  p.bn = 256;
+  p.bn = bn;
   p.out = act;
   p.ld_out = s.d_i;
   p.mask = const_cast<uint64_t *>(mask);
