@@ -159,7 +159,6 @@ def _num(s):
 # stage name -> the source files that define its kernel
 KERNEL_SOURCES = {
     "pred_h": ["predict_topk.cu"], "logits_topk": ["predict_topk.cu"],
-    "predict": ["predict_topk.cu"],
     "ffn": ["gather_ffn.cu"], "reduce": ["gather_ffn.cu"],
     "tc_h": ["tc_path.cu", "tc_util.cuh"], "tc_logits_topk": ["tc_path.cu", "tc_util.cuh"],
     "tc_gateup": ["tc_path.cu", "tc_util.cuh"], "tc_down": ["tc_path.cu", "tc_util.cuh"],
@@ -211,8 +210,6 @@ def stage_work(wl, T, union_channels):
            "flops": 6 * T * d_s * d}
     return {
         "pred_h": pred_h, "logits_topk": logits, "ffn": ffn,
-        "predict": {"bytes": pred_h["bytes"] + logits["bytes"] - T * r * 4,
-                    "flops": pred_h["flops"] + logits["flops"]},
         "reduce": {"bytes": T * d * e, "flops": 0},
         "tc_h": pred_h, "tc_logits_topk": logits,
         "tc_gateup": {"bytes": 2 * union_channels * d * e + T * d * e + T * d_i * e,
@@ -438,7 +435,7 @@ def run_sfn(args, rank, world, local):
 
     value = world * T * K / (elapsed_ms_max * 1e-3)
     # the path's algorithmic minimum: predictor weights, kept rows, x and y
-    step_bytes = sum(work[n]["bytes"] for n in ("predict", "ffn", "reduce"))
+    step_bytes = sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "ffn", "reduce"))
     step_flops = T * useful_flops_per_token(wl)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,

@@ -222,6 +222,23 @@ sfn_status sfn_sparse_ffn_forward_path(const void *x, const void *A, const void 
                                        int r, int bank, int k, sfn_path path, void *workspace,
                                        size_t workspace_bytes, sfn_stream_t stream);
 
+/*
+ * The pages' "Dense-4x" comparison (gist.science summary, "Resultaten": a
+ * dense model made 4x sparse post hoc from the activation amplitude).
+ * Reading: the standard SwiGLU FFN without a predictor -- act_j =
+ * silu(Wg[j].x) * (Wu[j].x) with silu(z) = z sigma(z); in every bank keep the
+ * k channels of largest |act_j| (ties to the lower index), zero the rest;
+ * y = sum_j act_j Wd[j, :].  bf16 in and out (x, Wg, Wu, Wd, y); mask, if not
+ * NULL, receives the kept channels.  Runs on the tensor cores: bank must be
+ * 64 and d, d_i multiples of 256 (else SFN_ERR_UNSUPPORTED).  Scratch: at
+ * least sfn_dense4x_workspace_bytes() bytes, 256-byte aligned.
+ */
+size_t sfn_dense4x_workspace_bytes(int64_t T, int d, int d_i, int bank, int k);
+sfn_status sfn_dense4x_forward(const void *x, const void *Wg, const void *Wu, const void *Wd,
+                               void *y, uint64_t *mask, int64_t T, int d, int d_i, int bank,
+                               int k, void *workspace, size_t workspace_bytes,
+                               sfn_stream_t stream);
+
 /* float32 twins of the two forward entry points. */
 sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
                                       const float *Wg, const float *Wu, const float *Wd,
@@ -253,7 +270,7 @@ enum {
   SFN_STAGE_TC_LOGITS_TOPK = 6, /* tensor cores: logits + fused top-k   */
   SFN_STAGE_TC_GATEUP = 7,    /* tensor cores: masked sigma(p) g u      */
   SFN_STAGE_TC_DOWN = 8,      /* tensor cores: y = act W_down           */
-  SFN_STAGE_PREDICT = 9,      /* h, logits and top-k in one cluster kernel */
+  SFN_STAGE_DENSE4X_GATEUP = 10, /* Dense-4x: silu(g) u + amplitude top-k */
   SFN_STAGE_COUNT = 16        /* room for the stage ids of this library */
 };
 sfn_status sfn_timing_begin(void);

@@ -64,6 +64,8 @@ def _open(path: str):
     lib.sfn_oracle_dense_then_mask.argtypes = [
         vp, ci, vp, vp, vp, ci, vp, ci, vp, ci, i64, ci, ci, ci, vp]
     lib.sfn_oracle_num_threads.restype = ci
+    lib.sfn_oracle_dense4x.argtypes = [vp, ci, vp, ci, vp, ci, vp, ci, i64, ci, ci, ci, ci, ci,
+                                       vp, vp, vp]
     return lib
 
 
@@ -190,6 +192,29 @@ def dense_then_mask(x, logits, mask, Wg, Wu, Wd, bank: int) -> np.ndarray:
                                        _ptr(ua), ud, _ptr(da), dd, T, d, d_i, bank,
                                        _ptr(y))
     return y
+
+
+def dense4x(x, Wg, Wu, Wd, bank: int, k: int, mask=None, want_act: bool = False):
+    """The Dense-4x comparison: SwiGLU act = silu(g) u, per bank keep the k
+    largest |act|, y = sum of kept act_j Wd[j].  Returns (y [T, d], mask) and,
+    with want_act, also act [T, d_i].  With ``mask`` given, that mask is
+    applied instead of the amplitude top-k."""
+    xa, xd = _arr(x)
+    ga, gd = _arr(Wg)
+    ua, ud = _arr(Wu)
+    da, dd = _arr(Wd)
+    T, d = xa.shape
+    d_i = ga.shape[0]
+    assert d_i % bank == 0 and 1 <= k <= bank <= 64
+    given = mask is not None
+    m = (np.ascontiguousarray(np.asarray(mask, dtype=np.uint64)).copy() if given
+         else np.empty((T, d_i // bank), np.uint64))
+    act = np.empty((T, d_i), np.float64) if want_act else None
+    y = np.empty((T, d), np.float64)
+    _load().sfn_oracle_dense4x(_ptr(xa), xd, _ptr(ga), gd, _ptr(ua), ud, _ptr(da), dd, T, d, d_i,
+                               bank, k, int(given), _ptr(m),
+                               _ptr(act) if want_act else None, _ptr(y))
+    return (y, m, act) if want_act else (y, m)
 
 
 def mask_to_bool(mask, bank: int) -> np.ndarray:

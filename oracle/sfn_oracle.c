@@ -204,6 +204,47 @@ void sfn_oracle_dense_then_mask(const void *x, int x_dt, const double *logits,
   }
 }
 
+/* The pages' "Dense-4x" comparison (gist.science summary, "Resultaten": a
+ * dense model with a naive 4x sparsity applied post hoc from the activation
+ * amplitude).  Reading: the standard SwiGLU FFN, act_j = silu(g_j) u_j with
+ * silu(z) = z sigma(z), g_j = Wg[j].x, u_j = Wu[j].x; in every bank keep the
+ * k channels of largest |act_j| (ties to the lower index, the same rule as
+ * sfn_oracle_bank_topk); y = sum_{kept j} act_j Wd[j, :].  No predictor.
+ * mask_io is [T][d_i/bank]: written, or (use_given_mask) read as the mask to
+ * apply; act_out, if not NULL, receives act [T][d_i]; y is [T][d]. */
+void sfn_oracle_dense4x(const void *x, int x_dt, const void *Wg, int Wg_dt, const void *Wu,
+                        int Wu_dt, const void *Wd, int Wd_dt, int64_t T, int d, int d_i,
+                        int bank, int k, int use_given_mask, uint64_t *mask_io, double *act_out,
+                        double *y) {
+  int nb = d_i / bank;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < T; ++t) {
+    double *act = (double *)malloc(sizeof(double) * (size_t)d_i);
+    double *amp = (double *)malloc(sizeof(double) * (size_t)d_i);
+    for (int j = 0; j < d_i; ++j) {
+      double g = 0.0, u = 0.0;
+      for (int n = 0; n < d; ++n) {
+        double xn = ld(x, x_dt, t * d + n);
+        g += ld(Wg, Wg_dt, (int64_t)j * d + n) * xn;
+        u += ld(Wu, Wu_dt, (int64_t)j * d + n) * xn;
+      }
+      act[j] = g * sfn_oracle_sigmoid(g) * u;
+      amp[j] = fabs(act[j]);
+    }
+    if (act_out)
+      for (int j = 0; j < d_i; ++j) act_out[t * d_i + j] = act[j];
+    if (!use_given_mask) sfn_oracle_bank_topk(amp, 1, d_i, bank, k, mask_io + t * nb);
+    double *yt = y + t * d;
+    for (int n = 0; n < d; ++n) yt[n] = 0.0;
+    for (int j = 0; j < d_i; ++j) {
+      if (!((mask_io[t * nb + j / bank] >> (j % bank)) & 1)) continue;
+      for (int n = 0; n < d; ++n) yt[n] += act[j] * ld(Wd, Wd_dt, (int64_t)j * d + n);
+    }
+    free(act);
+    free(amp);
+  }
+}
+
 /* Threads the OpenMP runtime will use (reported beside CPU timings). */
 int sfn_oracle_num_threads(void) {
 #ifdef _OPENMP

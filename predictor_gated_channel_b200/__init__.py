@@ -15,7 +15,7 @@ from __future__ import annotations
 from . import _capi
 from ._capi import SfnError
 
-__all__ = ["predict", "bank_topk", "sparse_ffn_forward", "workspace_bytes",
+__all__ = ["predict", "bank_topk", "sparse_ffn_forward", "dense4x_forward", "workspace_bytes",
            "kernel_launch_count", "SfnError"]
 
 
@@ -159,4 +159,29 @@ def sparse_ffn_forward(x, A, B, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None,
               else L.sfn_sparse_ffn_forward_f32_ws)
         _capi.check(fn(*args, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                        st), "sfn_sparse_ffn_forward_ws")
+    return y, mask
+
+
+def dense4x_forward(x, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None, mask=None,
+                    workspace=None, stream=None):
+    """The Dense-4x comparison (post-hoc amplitude top-k of the SwiGLU
+    activation, no predictor).  bf16.  Returns (y [T, d], mask int64)."""
+    torch = _torch()
+    for n, t in (("x", x), ("Wg", Wg), ("Wu", Wu), ("Wd", Wd)):
+        _dev(t, n)
+    T, d = x.shape
+    d_i = Wg.shape[0]
+    if y is None:
+        y = torch.empty((T, d), dtype=x.dtype, device=x.device)
+    if mask is None:
+        mask = torch.empty((T, max(d_i // max(bank, 1), 0)), dtype=torch.int64, device=x.device)
+    L = _capi.lib()
+    if workspace is None:
+        nbytes = int(L.sfn_dense4x_workspace_bytes(T, d, d_i, bank, k))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    _capi.check(L.sfn_dense4x_forward(x.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), Wd.data_ptr(),
+                                      y.data_ptr(), mask.data_ptr(), T, d, d_i, bank, k,
+                                      workspace.data_ptr(),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream_ptr(stream, x.device)), "sfn_dense4x_forward")
     return y, mask

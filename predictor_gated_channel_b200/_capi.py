@@ -42,6 +42,9 @@ SIGNATURES = {
     "sfn_sparse_ffn_forward_path": (_ci, _FWD + [_ci, _vp, _sz, _vp]),
     "sfn_sparse_ffn_forward_f32": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_f32_ws": (_ci, _FWD + [_vp, _sz, _vp]),
+    "sfn_dense4x_workspace_bytes": (_sz, [_i64, _ci, _ci, _ci, _ci]),
+    "sfn_dense4x_forward": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _ci, _ci, _ci, _ci, _vp,
+                                  _sz, _vp]),
     "sfn_timing_begin": (_ci, []),
     "sfn_device_errors": (_ci, [_vp, _ci]),
     "sfn_timing_end": (_ci, [_vp, _vp, _ci]),

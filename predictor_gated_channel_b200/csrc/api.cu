@@ -3,6 +3,8 @@
 // is enqueued, so an error status means nothing was written.
 #include <algorithm>
 #include <atomic>
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -74,6 +76,14 @@ int pow2_tokens(int64_t T, int cap) {
 }  // namespace
 
 void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+bool debug_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("SFN_DEBUG");
+    return v != nullptr && v[0] == '1';
+  }();
+  return on;
+}
 
 cudaError_t ensure_smem_limit(const void *kernel, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
@@ -150,6 +160,7 @@ GatherPlan plan_gather(const FwdShape &s) {
 using namespace sfn;
 
 namespace {
+thread_local const char *t_last_error = "no error";
 
 sfn_status check_shape(int64_t T, int d, int d_i, int r, int bank, int k) {
   if (T < 0 || d <= 0 || d_i <= 0 || r <= 0) return SFN_ERR_INVALID_VALUE;
@@ -182,8 +193,6 @@ FwdShape make_shape(int64_t T, int d, int d_i, int r, int bank, int k, bool bf16
   s.bf16 = bf16;
   return s;
 }
-
-thread_local const char *t_last_error = "no error";
 
 sfn_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SFN_OK;
@@ -235,12 +244,6 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
 
 // Fewest tokens for which the automatic choice takes the tensor-core path.
 constexpr int64_t kTcMinTokens = 1024;
-// Up to this many tokens the CUDA-core path computes the predictor and the
-// top-k in one cluster kernel (each cluster reads all of A once per token).
-constexpr int64_t kClusterPredictMaxTokens = 2;
-// Devices on which a cluster launch was refused (fall back to two kernels).
-std::atomic<bool> g_cluster_refused[64];
-
 bool use_tensor_path(const FwdShape &s, sfn_path path) {
   if (path == SFN_PATH_CUDA_CORE) return false;
   if (!tc_shape_ok(s)) return false;
@@ -344,6 +347,26 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     if (e == cudaSuccess) e = ef;
   }
   return cuda_status(e);
+}
+
+// Scratch of the Dense-4x comparison: act [T][d_i] bf16, a mask, and the
+// down GEMM's split-K partials.
+struct Dense4xPlan {
+  int ksplit;
+  size_t off_act, off_mask, off_part, total;
+};
+Dense4xPlan plan_dense4x(const FwdShape &s) {
+  Dense4xPlan p{};
+  p.ksplit = tc_down_splits(s, kPlanSms);
+  size_t off = 0;
+  p.off_act = off;
+  off = align_up(off + (size_t)s.T * s.d_i * 2, 256);
+  p.off_mask = off;
+  off = align_up(off + (size_t)s.T * s.n_banks * 8, 256);
+  p.off_part = off;
+  if (p.ksplit > 1) off = align_up(off + (size_t)s.T * p.ksplit * s.d * 4, 256);
+  p.total = off;
+  return p;
 }
 
 }  // namespace
@@ -495,6 +518,51 @@ sfn_status sfn_device_errors(unsigned *bits, int clear) {
   return SFN_OK;
 }
 
+size_t sfn_dense4x_workspace_bytes(int64_t T, int d, int d_i, int bank, int k) {
+  if (check_shape(T, d, d_i, 64, bank, k) != SFN_OK || T == 0) return 0;
+  if (check_limits(d, d_i, 64) != SFN_OK) return 0;
+  return plan_dense4x(make_shape(T, d, d_i, 64, bank, k, true)).total;
+}
+
+sfn_status sfn_dense4x_forward(const void *x, const void *Wg, const void *Wu, const void *Wd,
+                               void *y, uint64_t *mask, int64_t T, int d, int d_i, int bank,
+                               int k, void *ws, size_t ws_bytes, sfn_stream_t stream) {
+  sfn_status s0 = check_shape(T, d, d_i, 64, bank, k);
+  if (s0 != SFN_OK) return s0;
+  if ((s0 = check_limits(d, d_i, 64)) != SFN_OK) return s0;
+  if ((s0 = check_rows(d, 64, true)) != SFN_OK) return s0;
+  FwdShape s = make_shape(T, d, d_i, 64, bank, k, true);
+  if (!(bank == 64 && d % 256 == 0 && d_i % 256 == 0)) return SFN_ERR_UNSUPPORTED;
+  if (T == 0) return SFN_OK;
+  if (!x || !Wg || !Wu || !Wd || !y) return SFN_ERR_INVALID_VALUE;
+  if (!aligned(x, 16) || !aligned(Wg, 16) || !aligned(Wu, 16) || !aligned(Wd, 16) ||
+      !aligned(y, 16) || (mask && !aligned(mask, 8)))
+    return SFN_ERR_MISALIGNED;
+  const Dense4xPlan p = plan_dense4x(s);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < p.total) return SFN_ERR_WORKSPACE;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return SFN_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  char *w = static_cast<char *>(ws);
+  uint16_t *act = reinterpret_cast<uint16_t *>(w + p.off_act);
+  uint64_t *m = mask ? mask : reinterpret_cast<uint64_t *>(w + p.off_mask);
+  cudaError_t e = timed(SFN_STAGE_DENSE4X_GATEUP, st, [&] {
+    return launch_tc_dense4x_gateup(s, dev, x, Wg, Wu, m, act, st);
+  });
+  if (p.ksplit > 1) {
+    float *part = reinterpret_cast<float *>(w + p.off_part);
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_TC_DOWN, st,
+                [&] { return launch_tc_down(s, dev, act, Wd, part, p.ksplit, st); });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_REDUCE, st,
+                [&] { return launch_reduce_partials(s, p.ksplit, part, y, st); });
+  } else if (e == cudaSuccess) {
+    e = timed(SFN_STAGE_TC_DOWN, st, [&] { return launch_tc_down(s, dev, act, Wd, y, 1, st); });
+  }
+  return cuda_status(e);
+}
+
 const char *sfn_stage_name(int stage) {
   switch (stage) {
     case SFN_STAGE_PRED_H: return "pred_h";
@@ -505,7 +573,7 @@ const char *sfn_stage_name(int stage) {
     case SFN_STAGE_TC_LOGITS_TOPK: return "tc_logits_topk";
     case SFN_STAGE_TC_GATEUP: return "tc_gateup";
     case SFN_STAGE_TC_DOWN: return "tc_down";
-    case SFN_STAGE_PREDICT: return "predict";
+    case SFN_STAGE_DENSE4X_GATEUP: return "dense4x_gateup";
     case SFN_STAGE_BANK_TOPK: return "bank_topk";
   }
   return "unused";

@@ -278,202 +278,6 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
   }
 }
 
-// ------------------------------------------------------------ cluster fused
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-// Read a float from the shared memory of CTA `rank` of this cluster, at the
-// address `local` has in this CTA.
-__device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
-// Predictor and bank top-k in one kernel, for few tokens.  blockIdx.x =
-// token_group * n_banks + bank; clusters of CL consecutive banks.  CTA q of a
-// cluster computes rows [q * r / CL, (q + 1) * r / CL) of h = A x into its
-// shared memory; after a cluster barrier every CTA gathers the whole h over
-// distributed shared memory, then computes its bank's logits from its block
-// of B (bulk-copied in the prologue) and the bank's top-k, like
-// k_logits_topk.  A second cluster barrier keeps every CTA's slice of h alive
-// until all CTAs of the cluster have read it.
-template <class E, int TT>
-__global__ void __launch_bounds__(kThreads) k_predict_cluster(
-    const char *__restrict__ x, const char *__restrict__ A, const char *__restrict__ B,
-    uint64_t *__restrict__ mask, int *__restrict__ sel_idx, float *__restrict__ sel_sig,
-    int64_t T, int d, int d_i, int r, int bank, int k, int cl, unsigned *err) {
-  extern __shared__ float4 smem_f4[];
-  const uint32_t block_bytes = (uint32_t)bank * r * E::kBytes;
-  const int rows_per = r / cl;
-  unsigned char *bs = reinterpret_cast<unsigned char *>(smem_f4);         // [bank][r]
-  float *xs = reinterpret_cast<float *>(bs + block_bytes);                // [TT][d]
-  float *hpart = xs + TT * d;                                             // [TT][rows_per]
-  float *hs = hpart + TT * rows_per;                                      // [TT][r]
-  float *ps = hs + TT * r;                                                // [TT][64]
-  uint64_t *bbar = reinterpret_cast<uint64_t *>(ps + TT * 64);
-  const int n_banks = d_i / bank;
-  const int b = blockIdx.x % n_banks;
-  const int64_t t0 = (int64_t)(blockIdx.x / n_banks) * TT;
-  const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
-  const uint32_t q = cluster_ctarank();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const char *bblock = B + (int64_t)b * block_bytes;
-
-  if (threadIdx.x == 0) {
-    mbar_init(bbar, 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bbar, block_bytes);
-    for (uint32_t o = 0; o < block_bytes; o += 16384) {
-      const uint32_t n = block_bytes - o < 16384 ? block_bytes - o : 16384;
-      bulk_g2s(bs + o, bblock + o, n, bbar);
-    }
-  }
-  pdl_wait();
-  pdl_launch_dependents();
-  stage_rows<E, TT>(xs, x, t0, nt, d);
-  __syncthreads();
-
-  // phase 1: this CTA's rows of h, one warp per row
-  const int nchunk = d / E::kVec;
-  for (int lm = warp; lm < rows_per; lm += kWarps) {
-    const char *row = A + (int64_t)(q * rows_per + lm) * d * E::kBytes;
-    float acc[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-    for (int c0 = lane; c0 < nchunk; c0 += 32 * 16) {
-      uint4 v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int c = c0 + 32 * u;
-        v[u] = (c < nchunk) ? ld_stream16(row + (int64_t)c * 16) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int c = c0 + 32 * u;
-        if (c < nchunk) {
-          float a[E::kVec];
-          E::unpack(v[u], a);
-#pragma unroll
-          for (int t = 0; t < TT; ++t) {
-            const float *xr = xs + t * d + c * E::kVec;
-#pragma unroll
-            for (int e = 0; e < E::kVec; ++e) acc[t] = fmaf(a[e], xr[e], acc[t]);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const float v = warp_sum(acc[t]);
-      if (lane == 0) hpart[t * rows_per + lm] = v;
-    }
-  }
-  cluster_sync_all();
-  // phase 2: gather all of h from the cluster's CTAs
-  for (int i = threadIdx.x; i < TT * r; i += blockDim.x) {
-    const int t = i / r, m = i - t * r;
-    hs[i] = ld_dsmem_f32(hpart + t * rows_per + (m % rows_per), (uint32_t)(m / rows_per));
-  }
-  cluster_sync_all();
-  const bool ok = __syncthreads_and(mbar_wait(bbar, 0, err)) != 0;
-  if (!ok) {
-    if (threadIdx.x == 0) mbar_wait(bbar, 0, err);  // let in-flight copies land
-    return;
-  }
-
-  // phase 3: the bank's logits from shared memory, then its top-k
-  const int nchunk_r = r / E::kVec;
-  for (int jl0 = warp; jl0 < bank; jl0 += 4 * kWarps) {
-    float acc[4][TT];
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq)
-#pragma unroll
-      for (int t = 0; t < TT; ++t) acc[qq][t] = 0.f;
-    for (int c0 = lane; c0 < nchunk_r; c0 += 64) {
-      uint4 v[4][2];
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        const int jl = jl0 + qq * kWarps;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = c0 + 32 * u;
-          v[qq][u] = (jl < bank && c < nchunk_r)
-                         ? *reinterpret_cast<const uint4 *>(bs + ((size_t)jl * r + (size_t)c * E::kVec) * E::kBytes)
-                         : make_uint4(0, 0, 0, 0);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = c0 + 32 * u;
-        if (c < nchunk_r) {
-          float hv[TT][E::kVec];
-#pragma unroll
-          for (int t = 0; t < TT; ++t)
-#pragma unroll
-            for (int e = 0; e < E::kVec; e += 4) {
-              const float4 f = *reinterpret_cast<const float4 *>(hs + t * r + c * E::kVec + e);
-              hv[t][e] = f.x;
-              hv[t][e + 1] = f.y;
-              hv[t][e + 2] = f.z;
-              hv[t][e + 3] = f.w;
-            }
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            float w[E::kVec];
-            E::unpack(v[qq][u], w);
-#pragma unroll
-            for (int t = 0; t < TT; ++t)
-#pragma unroll
-              for (int e = 0; e < E::kVec; ++e) acc[qq][t] = fmaf(w[e], hv[t][e], acc[qq][t]);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq) {
-      const int jl = jl0 + qq * kWarps;
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        const float v = warp_sum(acc[qq][t]);
-        if (lane == 0 && jl < bank) ps[t * 64 + jl] = v;
-      }
-    }
-  }
-  __syncthreads();
-  const int d_s = n_banks * k;
-  for (int t = warp; t < nt; t += kWarps) {
-    const float p0 = (lane < bank) ? ps[t * 64 + lane] : 0.f;
-    const float p1 = (lane + 32 < bank) ? ps[t * 64 + lane + 32] : 0.f;
-    const uint64_t word = warp_bank_topk(order_key(p0), order_key(p1), bank, k);
-    const int64_t tg = t0 + t;
-    if (mask != nullptr && lane == 0) mask[tg * n_banks + b] = word;
-    int *idx_row = sel_idx + tg * d_s + b * k;
-    float *sig_row = sel_sig + tg * d_s + b * k;
-    if ((word >> lane) & 1ull) {
-      const int s_ = __popcll(word & ((1ull << lane) - 1ull));
-      idx_row[s_] = b * bank + lane;
-      sig_row[s_] = sigmoid_f32(p0);
-    }
-    if ((word >> (lane + 32)) & 1ull) {
-      const int s_ = __popcll(word & ((1ull << (lane + 32)) - 1ull));
-      idx_row[s_] = b * bank + lane + 32;
-      sig_row[s_] = sigmoid_f32(p1);
-    }
-  }
-}
-
 // Standalone top-k: one warp per (token, bank).
 __global__ void __launch_bounds__(kThreads) k_bank_topk(const float *__restrict__ logits,
                                                         uint64_t *__restrict__ mask,
@@ -578,60 +382,6 @@ cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const 
   if (topk)
     return logits_dispatch<EltF32, false, true>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
   return logits_dispatch<EltF32, true, false>(s, tt, h, B, logits, mask, sel_idx, sel_sig, err, st);
-}
-
-namespace {
-template <class E, int TT>
-cudaError_t predict_cluster_tt(const FwdShape &s, int cl, const void *x, const void *A,
-                               const void *B, uint64_t *mask, int *sel_idx, float *sel_sig,
-                               unsigned *err, cudaStream_t st) {
-  const size_t smem = (size_t)s.bank * s.r * E::kBytes +
-                      sizeof(float) * ((size_t)TT * s.d + (size_t)TT * (s.r / cl) +
-                                       (size_t)TT * s.r + (size_t)TT * 64) + 16;
-  auto kern = k_predict_cluster<E, TT>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e != cudaSuccess) return e;
-  const int64_t blocks = (int64_t)s.n_banks * ((s.T + TT - 1) / TT);
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)blocks);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = cl;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, kern, (const char *)x, (const char *)A, (const char *)B, mask,
-                         sel_idx, sel_sig, s.T, s.d, s.d_i, s.r, s.bank, s.k, cl, err);
-  count_launches(1);
-  return e;
-}
-}  // namespace
-
-int predict_cluster_size(const FwdShape &s) {
-  // bf16 or f32; the bank block of B, x rows and h fit beside each other
-  const size_t elt = s.bf16 ? 2 : 4;
-  if ((size_t)s.bank * s.r * elt > kMaxBBlock || (size_t)s.d * 4 > 32768) return 0;
-  for (int cl : {16, 8, 4, 2}) {
-    if (s.n_banks % cl == 0 && s.r % cl == 0) return cl;
-  }
-  return 0;
-}
-
-cudaError_t launch_predict_cluster(const FwdShape &s, int cl, const void *x, const void *A,
-                                   const void *B, uint64_t *mask, int *sel_idx,
-                                   float *sel_sig, unsigned *err, cudaStream_t st) {
-  // one token per CTA keeps the staged x small; more tokens are more CTAs
-  if (s.bf16) return predict_cluster_tt<EltBF16, 1>(s, cl, x, A, B, mask, sel_idx, sel_sig, err, st);
-  return predict_cluster_tt<EltF32, 1>(s, cl, x, A, B, mask, sel_idx, sel_sig, err, st);
 }
 
 cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,

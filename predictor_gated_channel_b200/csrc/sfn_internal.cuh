@@ -120,6 +120,9 @@ bool device_info(DeviceInfo *out);
 
 void count_launches(uint64_t n);
 
+// SFN_DEBUG=1 in the environment: diagnostic messages on stderr.
+bool debug_enabled();
+
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
@@ -173,11 +176,7 @@ cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const 
                                unsigned *err, cudaStream_t st);
 cudaError_t launch_bank_topk(const float *logits, uint64_t *mask, int64_t T, int d_i,
                              int bank, int k, cudaStream_t st);
-// Cluster size for the fused predictor + top-k kernel (0: not applicable).
-int predict_cluster_size(const FwdShape &s);
-cudaError_t launch_predict_cluster(const FwdShape &s, int cl, const void *x, const void *A,
-                                   const void *B, uint64_t *mask, int *sel_idx,
-                                   float *sel_sig, unsigned *err, cudaStream_t st);
+
 bool ffn_shape_ok(const FwdShape &s);
 int ffn_ctas_per_token(const FwdShape &s, int num_sms);
 cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
@@ -207,6 +206,9 @@ cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uin
 cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
                              const void *Wg, const void *Wu, const uint64_t *mask,
                              const float *sig, uint16_t *act, cudaStream_t st);
+cudaError_t launch_tc_dense4x_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
+                                     const void *Wg, const void *Wu, uint64_t *mask,
+                                     uint16_t *act, cudaStream_t st);
 cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
                            const void *Wd, void *y, int ksplit, cudaStream_t st);
 

@@ -47,7 +47,14 @@ constexpr int kAccCols = 256;                  // TMEM columns per accumulator
 constexpr size_t kMaxDynSmem = 232448;            // 227 KB per CTA on sm_100
 constexpr int kGroupM = 8;                     // tile rasterisation group
 
-enum : int { kEpiHSplit = 0, kEpiLogits = 1, kEpiTopk = 2, kEpiGateUp = 3, kEpiDown = 4 };
+enum : int {
+  kEpiHSplit = 0,
+  kEpiLogits = 1,
+  kEpiTopk = 2,
+  kEpiGateUp = 3,
+  kEpiDown = 4,
+  kEpiDense4x = 5  // gate/up GEMM of the post-hoc amplitude top-k comparison
+};
 
 struct TcParams {
   int64_t T;
@@ -69,6 +76,7 @@ template <int kEpi>
 struct EpiTraits {
   static constexpr int kNumA = (kEpi == kEpiLogits || kEpi == kEpiTopk) ? 2 : 1;
   static constexpr bool kBMnMajor = (kEpi == kEpiDown);
+  static constexpr bool kGateUpB = (kEpi == kEpiGateUp || kEpi == kEpiDense4x);
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &mb,
@@ -160,6 +168,32 @@ __device__ __forceinline__ float sigmoid_fast(float z) {
 
 constexpr int kStageRow = 65;  // floats per epilogue thread row (k <= 64, padded)
 
+// k-th largest of 64 order keys (s is reordered), and the number of keys
+// strictly above it.
+__device__ __forceinline__ void keys_threshold(uint32_t (&s)[64], int k, uint32_t &tau, int &gt) {
+  gt = 0;
+  if (k == 16) {
+    BitonicSort<0, 16, 2>::run(s);
+    BitonicSort<16, 16, 2>::run(s);
+    BitonicSort<32, 16, 2>::run(s);
+    BitonicSort<48, 16, 2>::run(s);
+    merge_top16<0, 16>(s);
+    merge_top16<32, 48>(s);
+    tau = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tau = min(tau, max(s[i], s[47 - i]));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) gt += max(s[i], s[47 - i]) > tau;
+  } else {
+    BitonicSort<0, 64, 2>::run(s);
+    tau = s[0];
+#pragma unroll
+    for (int i = 1; i < 64; ++i) tau = (i == k - 1) ? s[i] : tau;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) gt += s[i] > tau;
+  }
+}
+
 // k-th largest order key of the 64 logits held in TMEM columns
 // [taddr, taddr + 64) of this thread's row, and the number of keys strictly
 // above it.
@@ -240,7 +274,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (lane == 0) {
       prefetch_tmap(&tA);
       prefetch_tmap(&tB);
-      if (kEpi == kEpiGateUp) prefetch_tmap(&tB2);
+      if (Tr::kGateUpB) prefetch_tmap(&tB2);
       uint32_t it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < total && ok; unit += gridDim.x) {
@@ -258,7 +292,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           mbar_arrive_expect_tx(&full[s], p.stage_bytes);
           tma_load_2d(a, &tA, kb * kBK, mb * kBM, &full[s]);
           if (Tr::kNumA == 2) tma_load_2d(a + kTileA, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
-          if (kEpi == kEpiGateUp) {
+          if (Tr::kGateUpB) {
             tma_load_2d(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
             tma_load_2d(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
           } else if (kEpi == kEpiDown) {
@@ -470,6 +504,67 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
         }
       }
+      if (kEpi == kEpiDense4x) {
+        // act = silu(g) u for every channel; per bank keep the k largest
+        // |act| (ties to the lower channel), zero the rest; bf16 out
+        uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
+        const int half_n = p.bn / 2;
+        for (int h = 0; h < half_n / 64; ++h) {
+          const int bank = nb * (half_n / 64) + h;
+          // pass 1: order keys of |act| for the 64 channels, then the threshold
+          uint32_t keys[64];
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t g[32], u[32];
+            tmem_ld_32x32b_x32(taddr + h * 64 + c0, g);
+            tmem_ld_32x32b_x32(taddr + half_n + h * 64 + c0, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float gv = __uint_as_float(g[i]);
+              keys[c0 + i] = order_key(fabsf(gv * sigmoid_fast(gv) * __uint_as_float(u[i])));
+            }
+          }
+          uint32_t tau;
+          int gt;
+          keys_threshold(keys, p.k, tau, gt);
+          const int need = p.k - gt;
+          int eq = 0;
+          uint32_t bits[2] = {0u, 0u};
+          // pass 2: recompute act half a bank at a time, keep or zero, store
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t g[32], u[32];
+            tmem_ld_32x32b_x32(taddr + h * 64 + c0, g);
+            tmem_ld_32x32b_x32(taddr + half_n + h * 64 + c0, u);
+            tmem_ld_wait();
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              float o2[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const float gv = __uint_as_float(g[i + e]);
+                const float a = gv * sigmoid_fast(gv) * __uint_as_float(u[i + e]);
+                const uint32_t key = order_key(fabsf(a));
+                const bool take = (key > tau) | ((key == tau) & (eq < need));
+                eq += (key == tau);
+                bits[c0 >> 5] |= (uint32_t)take << (i + e);
+                o2[e] = take ? a : 0.f;
+              }
+              packed[i / 2] = pack_bf16x2(o2[0], o2[1]);
+            }
+            if (valid) {
+              uint4 *dst = reinterpret_cast<uint4 *>(out + t * p.ld_out + bank * 64 + c0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
+                                    packed[4 * i + 3]);
+            }
+          }
+          if (valid) p.mask[t * p.n_banks + bank] = ((uint64_t)bits[1] << 32) | bits[0];
+        }
+      }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -679,6 +774,28 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
   p.mask = const_cast<uint64_t *>(mask);
   p.sig = const_cast<float *>(sig);
   return launch_tc<kEpiGateUp>(mX, mG, mU, p, dev.num_sms, st);
+}
+
+// Dense-4x comparison, first GEMM: [G | U] = X [Wg; Wu]^T -> act =
+// silu(g) u kept where |act| is among the k largest of its bank, 0 elsewhere.
+cudaError_t launch_tc_dense4x_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
+                                     const void *Wg, const void *Wu, uint64_t *mask,
+                                     uint16_t *act, cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  const int tiles_m = (int)((s.T + kBM - 1) / kBM);
+  const int bn = 2 * pick_bn(tiles_m, s.d_i, {128, 64}, dev.num_sms);
+  CUtensorMap mX, mG, mU;
+  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mG, Wg, s.d, s.d_i, 64, bn / 2) ||
+      !make_map(&mU, Wu, s.d, s.d_i, 64, bn / 2))
+    return cudaErrorInvalidValue;
+  TcParams p = base_params(s, dev);
+  p.tiles_n = s.d_i / (bn / 2);
+  p.k_blocks = s.d / kBK;
+  p.bn = bn;
+  p.out = act;
+  p.ld_out = s.d_i;
+  p.mask = mask;
+  return launch_tc<kEpiDense4x>(mX, mG, mU, p, dev.num_sms, st);
 }
 
 // G4: Y = act Wd, with Wd [d_i][d] read as an MN-major B operand.  With

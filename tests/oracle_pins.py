@@ -248,9 +248,24 @@ def pin_forward_bf16_widening():
     assert np.array_equal(p1, p2) and np.array_equal(m1, m2) and np.array_equal(y1, y2)
 
 
+def pin_dense4x():
+    """Dense-4x against numpy: amplitudes |silu(g) u|, the stable-sort top-k
+    of them, the masked SwiGLU FFN; k = bank is the dense SwiGLU FFN."""
+    rng = _rng(11)
+    x, A, B, Wg, Wu, Wd = _layer(rng, d=36, d_i=128, r=4)
+    g = x @ Wg.T
+    u = x @ Wu.T
+    act = g * expit(g) * u
+    for bank, k in [(64, 16), (32, 5), (64, 64)]:
+        y, m = oracle.dense4x(x, Wg, Wu, Wd, bank, k)
+        assert (m == _mask_by_stable_sort(np.abs(act), bank, k)).all()
+        keep = oracle.mask_to_bool(m, bank).astype(np.float64)
+        assert np.allclose(y, ((Wd.T) @ (keep * act).T).T, rtol=1e-11, atol=1e-12)
+
+
 ALL_PINS = [
     pin_topk_golden, pin_topk_popcount, pin_topk_stable_sort, pin_topk_brute_force,
     pin_predict_matmul, pin_predict_selector, pin_predict_integer_exact, pin_sigmoid,
     pin_forward_golden, pin_forward_k_equals_bank, pin_forward_masked_dense,
-    pin_forward_invariants, pin_forward_bf16_widening,
+    pin_forward_invariants, pin_forward_bf16_widening, pin_dense4x,
 ]

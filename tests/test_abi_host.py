@@ -126,3 +126,37 @@ def test_no_cpu_fallback():
         pytest.skip("a GPU is present")
     sfn_build.build()
     assert fwd(_capi.lib()) == _capi.SFN_ERR_CUDA
+
+
+def test_dense4x_validation(L):
+    need = L.sfn_dense4x_workspace_bytes(4, 4096, 14336, 64, 16)
+    assert need > 0 and need % 256 == 0
+    assert L.sfn_dense4x_workspace_bytes(0, 4096, 14336, 64, 16) == 0
+    args = [FAKE] * 5 + [None]
+    # shapes the tensor cores do not cover
+    assert L.sfn_dense4x_forward(*args, 4, 4096, 14336, 32, 8, FAKE, need, None) == \
+        _capi.SFN_ERR_UNSUPPORTED
+    assert L.sfn_dense4x_forward(*args, 4, 4160, 14336, 64, 16, FAKE, need, None) == \
+        _capi.SFN_ERR_UNSUPPORTED
+    assert L.sfn_dense4x_forward(*args, 4, 4096, 14336, 64, 0, FAKE, need, None) == \
+        _capi.SFN_ERR_INVALID_VALUE
+    assert L.sfn_dense4x_forward(*args, 0, 4096, 14336, 64, 16, None, 0, None) == _capi.SFN_OK
+    assert L.sfn_dense4x_forward(*args, 4, 4096, 14336, 64, 16, FAKE, 256, None) == \
+        _capi.SFN_ERR_WORKSPACE
+    p = [FAKE] * 5
+    p[0] = None
+    assert L.sfn_dense4x_forward(*p, None, 4, 4096, 14336, 64, 16, FAKE, need, None) == \
+        _capi.SFN_ERR_INVALID_VALUE
+    p[0] = FAKE + 8
+    assert L.sfn_dense4x_forward(*p, None, 4, 4096, 14336, 64, 16, FAKE, need, None) == \
+        _capi.SFN_ERR_MISALIGNED
+
+
+def test_path_selector_validation(L):
+    args = [FAKE] * 7 + [None, 4, 4096, 14336, 448, 64, 16]
+    need = L.sfn_workspace_bytes(4, 4096, 14336, 448, 64, 16, 0)
+    assert L.sfn_sparse_ffn_forward_path(*args, 7, FAKE, need, None) == _capi.SFN_ERR_INVALID_VALUE
+    bad = [FAKE] * 7 + [None, 4, 4096, 14336, 448, 32, 8]
+    assert L.sfn_sparse_ffn_forward_path(*bad, _capi.SFN_PATH_TENSOR, FAKE, need, None) == \
+        _capi.SFN_ERR_UNSUPPORTED
+    assert L.sfn_last_error_string() is not None

@@ -279,3 +279,24 @@ def test_tensor_path_rejects_unsupported(full_layer):
     with pytest.raises(sfn.SfnError):
         sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"],
                                bank=32, k=8, path="tensor")
+
+
+# ------------------------------------------------------------------ Dense-4x
+
+@pytest.mark.parametrize("T", [1, 64, 300])
+def test_dense4x_against_oracle(T, full_layer):
+    """The Dense-4x comparison on the tensor cores: the mask may differ from
+    the oracle's only at near-ties of the amplitude |silu(g) u|; y matches the
+    oracle applied with the GPU's own mask."""
+    wl, host, dev = full_layer
+    x = make_tokens(wl, T=T, seed=300 + T)
+    y, mask = sfn.dense4x_forward(x.to(DEV), dev["Wg"], dev["Wu"], dev["Wd"])
+    torch.cuda.synchronize()
+    rows = np.arange(T) if T <= 64 else np.arange(0, T, 11)
+    xs = x[torch.as_tensor(rows)]
+    _, _, act = oracle.dense4x(xs, host["Wg"], host["Wu"], host["Wd"], 64, 16, want_act=True)
+    gm = parity.to_u64(mask)[rows]
+    parity.check_mask(gm, np.abs(act), 64, 16)
+    y_ref, _ = oracle.dense4x(xs, host["Wg"], host["Wu"], host["Wd"], 64, 16, mask=gm)
+    err = parity.y_error(y.float().cpu().numpy()[rows], y_ref)
+    assert err <= parity.Y_TOL["bf16"], err

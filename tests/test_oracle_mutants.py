@@ -32,6 +32,9 @@ MUTANTS = {
                               "ld(A, A_dt, (int64_t)m * d + n) * ld(x, x_dt, n);"),
     "predictor_skips_last_rank": ("for (int m = 0; m < r; ++m) s += ld(B",
                                   "for (int m = 0; m < r - 1; ++m) s += ld(B"),
+    "dense4x_amplitude_signed": ("amp[j] = fabs(act[j]);", "amp[j] = act[j];"),
+    "dense4x_gate_not_silu": ("act[j] = g * sfn_oracle_sigmoid(g) * u;",
+                              "act[j] = sfn_oracle_sigmoid(g) * u;"),
 }
 
 
