@@ -230,7 +230,9 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
   } else {
     GatherPlan p = plan_gather(s);
     float *h = static_cast<float *>(scratch);
-    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, false, st); });
+    const size_t b_bytes = (size_t)s.d_i * s.r * (s.bf16 ? 2 : 4);
+    e = timed(SFN_STAGE_PRED_H, st,
+              [&] { return launch_pred_h(s, p.tt_h, x, A, h, false, st, B, b_bytes); });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
         return launch_logits_topk(s, p.tt_p, h, B, logits, nullptr, nullptr, nullptr, dev.err,
@@ -329,7 +331,9 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     int *sel_idx = reinterpret_cast<int *>(w + p.off_idx);
     float *sel_sig = reinterpret_cast<float *>(w + p.off_sig);
     float *partial = reinterpret_cast<float *>(w + p.off_part);
-    e = timed(SFN_STAGE_PRED_H, st, [&] { return launch_pred_h(s, p.tt_h, x, A, h, false, st); });
+    const size_t b_bytes = (size_t)s.d_i * s.r * (s.bf16 ? 2 : 4);
+    e = timed(SFN_STAGE_PRED_H, st,
+              [&] { return launch_pred_h(s, p.tt_h, x, A, h, false, st, B, b_bytes); });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
         return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, dev.err, st);
@@ -340,7 +344,7 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
       });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_REDUCE, st,
-                [&] { return launch_reduce_partials(s, p.cpt, partial, y, st); });
+                [&] { return launch_reduce_partials(s, p.cpt, partial, y, st, ReduceOut::kYLast); });
   }
   if (own_ws) {
     cudaError_t ef = cudaFreeAsync(ws, st);

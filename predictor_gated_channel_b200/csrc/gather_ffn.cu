@@ -30,7 +30,9 @@ namespace {
 constexpr int kMaxStages = 8;   // ring stages = gate/up warps (one each)
 constexpr int kDownWarps = 8;   // output column eighths
 constexpr int kMaxChunks = 4;   // 16-byte column chunks per down lane
-constexpr size_t kRingBudget = 192 * 1024;
+// 7 stages of 24 KB rows (d = 4096, bf16): leaves room on the SM for the
+// next call's h kernel, which prefetches the predictor weights meanwhile
+constexpr size_t kRingBudget = 168 * 1024;
 constexpr int kMaxSlotsPerCta = 1024;
 constexpr uint32_t kMaxXBytes = 16384;  // one token row of x staged in smem
 constexpr int kReduceThreads = 256;
@@ -97,14 +99,25 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
   }
   pdl_wait();  // sel_idx and sel_sig come from the previous kernel
   pdl_launch_dependents();
-  // stage this CTA's kept channel ids, their sigma(p) and the token's x
-  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-    idx_s[i] = sel_idx[f0 + i];
-    sig_s[i] = sel_sig[f0 + i];
-  }
+  // stage this CTA's kept channel ids, their sigma(p) and the token's x;
+  // each thread issues its loads before its stores (one round trip)
   const uint32_t row = L.row_bytes;
-  for (uint32_t o = threadIdx.x * 16; o < row; o += blockDim.x * 16)
-    *reinterpret_cast<uint4 *>(x_s + o) = ld_nc16(x + t * row + o);
+  const int nx = (int)(row / 16);
+  for (int i = threadIdx.x; i < cnt || i < nx; i += blockDim.x) {
+    int j = 0;
+    float sg = 0.f;
+    uint4 xv = make_uint4(0, 0, 0, 0);
+    if (i < cnt) {
+      j = sel_idx[f0 + i];
+      sg = sel_sig[f0 + i];
+    }
+    if (i < nx) xv = ld_nc16(x + t * row + (size_t)i * 16);
+    if (i < cnt) {
+      idx_s[i] = j;
+      sig_s[i] = sg;
+    }
+    if (i < nx) *reinterpret_cast<uint4 *>(x_s + (size_t)i * 16) = xv;
+  }
   __syncthreads();
 
   if (warp == S + kDownWarps) {
@@ -113,6 +126,9 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
     // ...: several independent issuers keep more row fetches in flight than
     // one thread issuing every copy in turn.
     const int st = lane;
+    // kept rows are read once: evict them from L2 first, ahead of the next
+    // call's predictor weights that its first kernel prefetches meanwhile
+    const uint64_t once = make_evict_first_policy();
     if (st < S) {
       int issued = 0;
       for (int n = st; n < cnt; n += S) {
@@ -123,10 +139,10 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
         const int64_t j = idx_s[n];
         unsigned char *gdst = gu_ring + (size_t)st * 2 * row;
         mbar_arrive_expect_tx(&gu_full[st], 2 * row);
-        bulk_g2s(gdst, Wg + j * row, row, &gu_full[st]);
-        bulk_g2s(gdst + row, Wu + j * row, row, &gu_full[st]);
+        bulk_g2s_hint(gdst, Wg + j * row, row, &gu_full[st], once);
+        bulk_g2s_hint(gdst + row, Wu + j * row, row, &gu_full[st], once);
         mbar_arrive_expect_tx(&d_full[st], row);
-        bulk_g2s(d_ring + (size_t)st * row, Wd + j * row, row, &d_full[st]);
+        bulk_g2s_hint(d_ring + (size_t)st * row, Wd + j * row, row, &d_full[st], once);
         issued = use + 1;
       }
       // never leave while a copy may still be landing in shared memory
@@ -215,7 +231,7 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
 // quad q): group g sums partials c = g, g + G, ...; the G group sums are then
 // added in group order.  kOut: 0 = float32 out, 1 = bf16 out, 2 = bf16 hi/lo
 // halves of h ([T][2n]: hi at column j, lo = bf16(sum - hi) at n + j).
-template <int C, int kOut>
+template <int C, int kOut, bool kEarly>
 __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
     const float *__restrict__ partial, void *__restrict__ out, int n, int cpt) {
   constexpr int Q = C / 4;                // float4 quads per slice
@@ -226,12 +242,16 @@ __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
   const int c0 = (blockIdx.x % slices) * C;
   const int g = threadIdx.x / Q, q = threadIdx.x % Q;
   const int col = c0 + q * 4;
+  // kEarly (last kernel of a forward call): the next call's first kernel may
+  // start at once; it reads only weights before its own griddepcontrol.wait,
+  // which returns after this kernel -- and so everything before it -- is done
+  if (kEarly) pdl_launch_dependents();
   pdl_wait();
-  pdl_launch_dependents();
+  if (!kEarly) pdl_launch_dependents();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (col < n) {
     const float *p = partial + t * cpt * (int64_t)n + col;
-#pragma unroll 4
+#pragma unroll 8
     for (int c = g; c < cpt; c += G) {
       const float4 v = *reinterpret_cast<const float4 *>(p + (int64_t)c * n);
       acc.x += v.x;
@@ -327,9 +347,15 @@ cudaError_t reduce_c(const FwdShape &s, int n, int cpt, const float *partial, vo
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const dim3 grid((unsigned)blocks), block(kReduceThreads);
   if (kind == ReduceOut::kSplitH)
-    return launch_pdl(k_reduce_partials<C, 2>, grid, block, 0, st, partial, out, n, cpt);
-  if (s.bf16) return launch_pdl(k_reduce_partials<C, 1>, grid, block, 0, st, partial, out, n, cpt);
-  return launch_pdl(k_reduce_partials<C, 0>, grid, block, 0, st, partial, out, n, cpt);
+    return launch_pdl(k_reduce_partials<C, 2, false>, grid, block, 0, st, partial, out, n, cpt);
+  if (kind == ReduceOut::kYLast) {
+    if (s.bf16)
+      return launch_pdl(k_reduce_partials<C, 1, true>, grid, block, 0, st, partial, out, n, cpt);
+    return launch_pdl(k_reduce_partials<C, 0, true>, grid, block, 0, st, partial, out, n, cpt);
+  }
+  if (s.bf16)
+    return launch_pdl(k_reduce_partials<C, 1, false>, grid, block, 0, st, partial, out, n, cpt);
+  return launch_pdl(k_reduce_partials<C, 0, false>, grid, block, 0, st, partial, out, n, cpt);
 }
 
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,

@@ -33,25 +33,35 @@ constexpr int kWarpsH = kThreadsH / 32;
 constexpr uint32_t kMaxBBlock = 96 * 1024;  // bank block of B staged in smem
 
 // Stage TT token rows of x (element type E) into shared memory as float;
-// rows past the end of the batch are zero.
+// rows past the end of the batch are zero.  Each thread issues up to 8 of its
+// loads before any store, so a row costs one memory round trip.
 template <class E, int TT>
 __device__ __forceinline__ void stage_rows(float *xs, const char *x, int64_t t0, int nt,
                                            int d) {
   const int nchunk = d / E::kVec;
-  for (int i = threadIdx.x; i < TT * nchunk; i += blockDim.x) {
-    const int t = i / nchunk, c = i - t * nchunk;
-    float f[E::kVec];
-    if (t < nt) {
-      const uint4 v = ld_nc16(x + ((t0 + t) * (int64_t)d + (int64_t)c * E::kVec) * E::kBytes);
-      E::unpack(v, f);
-    } else {
+  const int total = TT * nchunk;
+  for (int i0 = threadIdx.x; i0 < total; i0 += 8 * blockDim.x) {
+    uint4 v[8];
 #pragma unroll
-      for (int e = 0; e < E::kVec; ++e) f[e] = 0.f;
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      const int t = i / nchunk, c = i - t * nchunk;
+      v[u] = (i < total && t < nt)
+                 ? ld_nc16(x + ((t0 + t) * (int64_t)d + (int64_t)c * E::kVec) * E::kBytes)
+                 : make_uint4(0, 0, 0, 0);
     }
-    float4 *dst = reinterpret_cast<float4 *>(xs + t * d + c * E::kVec);
 #pragma unroll
-    for (int e = 0; e < E::kVec / 4; ++e)
-      dst[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < total) {
+        float f[E::kVec];
+        E::unpack(v[u], f);
+        float4 *dst = reinterpret_cast<float4 *>(xs + (size_t)i * E::kVec);
+#pragma unroll
+        for (int e = 0; e < E::kVec / 4; ++e)
+          dst[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+      }
+    }
   }
 }
 
@@ -60,18 +70,28 @@ __device__ __forceinline__ void stage_rows(float *xs, const char *x, int64_t t0,
 // kSplitOut: instead of fp32 h [T][r], write h as two bf16 halves
 // hi = bf16(h), lo = bf16(h - hi) into [T][2r] (hi first), the operand form
 // of the tensor-core logits GEMM.
+// pf (may be null): pf_bytes of weights the next kernel reads (the rows of
+// B), prefetched into L2 by the first token group's CTAs in the prologue,
+// together with this CTA's rows of A, before griddepcontrol.wait.
 template <class E, int TT, bool kSplitOut>
 __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x,
                                                       const char *__restrict__ A,
                                                       void *__restrict__ h_out, int64_t T,
-                                                      int d, int r) {
+                                                      int d, int r, const char *__restrict__ pf,
+                                                      int64_t pf_bytes) {
   extern __shared__ float4 smem_f4[];
   float *xs = reinterpret_cast<float *>(smem_f4);
   const int row_blocks = (r + kWarpsH - 1) / kWarpsH;
   const int64_t tg = blockIdx.x / row_blocks;
   const int rb = blockIdx.x % row_blocks;
-  pdl_wait();
-  pdl_launch_dependents();
+  if (pf != nullptr && tg == 0 && threadIdx.x < 32) {
+    constexpr int64_t kPiece = 16384;
+    const int64_t share = (pf_bytes / row_blocks + kPiece - 1) / kPiece * kPiece;
+    const int64_t b0 = rb * share;
+    const int64_t b1 = (b0 + share < pf_bytes) ? b0 + share : pf_bytes;
+    for (int64_t o = b0 + threadIdx.x * kPiece; o < b1; o += 32 * kPiece)
+      prefetch_l2(pf + o, (uint32_t)(b1 - o < kPiece ? b1 - o : kPiece));
+  }
 
   const int64_t t0 = tg * TT;
   const int nt = (T - t0 < TT) ? (int)(T - t0) : TT;
@@ -82,14 +102,16 @@ __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
-  // The row's first 16 loads per lane go out before x is staged, so the
-  // weight fetch overlaps the staging (8 KB bf16 rows: the whole row).
+  // The row's first 16 loads per lane go out before the wait and before x
+  // is staged (8 KB bf16 rows: the whole row).
   uint4 v[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
     const int c = lane + 32 * u;
     v[u] = (m < r && c < nchunk) ? ld_stream16(row + (int64_t)c * 16) : make_uint4(0, 0, 0, 0);
   }
+  pdl_wait();  // x may come from earlier work on the stream
+  pdl_launch_dependents();
   stage_rows<E, TT>(xs, x, t0, nt, d);
   __syncthreads();
   if (m >= r) return;
@@ -173,9 +195,23 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
   }
   pdl_wait();
   pdl_launch_dependents();
-  for (int i = threadIdx.x; i < TT * r; i += blockDim.x) {
-    const int t = i / r;
-    hs[i] = (t < nt) ? h[(t0 + t) * r + (i - t * r)] : 0.f;
+  // h rows for the token group, float4 at a time (r % 4 == 0), all loads of
+  // a thread issued before its stores
+  for (int i0 = threadIdx.x; i0 < TT * r / 4; i0 += 4 * blockDim.x) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      const int t = 4 * i / r;
+      v[u] = (i < TT * r / 4 && t < nt)
+                 ? *reinterpret_cast<const float4 *>(h + (t0 + t) * r + (4 * i - t * r))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < TT * r / 4) reinterpret_cast<float4 *>(hs)[i] = v[u];
+    }
   }
   __syncthreads();
   bool ok = true;
@@ -294,7 +330,7 @@ __global__ void __launch_bounds__(kThreads) k_bank_topk(const float *__restrict_
 
 template <class E, int TT, bool SPLIT>
 cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, void *h,
-                      cudaStream_t st) {
+                      const void *pf, size_t pf_bytes, cudaStream_t st) {
   const size_t smem = (size_t)TT * s.d * sizeof(float);
   auto kern = k_pred_h<E, TT, SPLIT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
@@ -302,7 +338,7 @@ cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, void *h,
   const int64_t blocks = (int64_t)((s.r + kWarpsH - 1) / kWarpsH) * ((s.T + TT - 1) / TT);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   e = launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreadsH), smem, st, (const char *)x,
-                 (const char *)A, h, s.T, s.d, s.r);
+                 (const char *)A, h, s.T, s.d, s.r, (const char *)pf, (int64_t)pf_bytes);
   count_launches(1);
   return e;
 }
@@ -344,10 +380,11 @@ cudaError_t logits_dispatch(const FwdShape &s, int tt, const float *h, const voi
 }  // namespace
 
 cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, void *h,
-                          bool split_out, cudaStream_t st) {
-#define SFN_PH(ELT, TTV)                                               \
-  return split_out ? pred_h_tt<ELT, TTV, true>(s, x, A, h, st) \
-                   : pred_h_tt<ELT, TTV, false>(s, x, A, h, st)
+                          bool split_out, cudaStream_t st, const void *prefetch,
+                          size_t prefetch_bytes) {
+#define SFN_PH(ELT, TTV)                                                                     \
+  return split_out ? pred_h_tt<ELT, TTV, true>(s, x, A, h, prefetch, prefetch_bytes, st) \
+                   : pred_h_tt<ELT, TTV, false>(s, x, A, h, prefetch, prefetch_bytes, st)
   if (s.bf16) {
     switch (tt) {
       case 1: SFN_PH(EltBF16, 1);

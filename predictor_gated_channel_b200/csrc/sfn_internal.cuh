@@ -169,8 +169,11 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // Launchers (enqueue only; return the launch status).
+// prefetch (may be null): prefetch_bytes of weights (a multiple of 16) that
+// the next kernel reads, brought into L2 in the h kernel's prologue.
 cudaError_t launch_pred_h(const FwdShape &s, int tt, const void *x, const void *A, void *h,
-                          bool split_out, cudaStream_t st);
+                          bool split_out, cudaStream_t st, const void *prefetch = nullptr,
+                          size_t prefetch_bytes = 0);
 cudaError_t launch_logits_topk(const FwdShape &s, int tt, const float *h, const void *B,
                                float *logits, uint64_t *mask, int *sel_idx, float *sel_sig,
                                unsigned *err, cudaStream_t st);
@@ -183,8 +186,10 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
                        const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
                        float *partial, unsigned *err, cudaStream_t st);
 // Output of k_reduce_partials: y in the call's element type, or the bf16
-// hi/lo halves of h ([T][2r], "split").
-enum class ReduceOut { kY, kSplitH };
+// hi/lo halves of h ([T][2r], "split").  kYLast: y, from the last kernel of
+// a call on the CUDA-core path, which lets the stream's next kernel start
+// its (weights-only) prologue at once.
+enum class ReduceOut { kY, kYLast, kSplitH };
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
                                    cudaStream_t st, ReduceOut kind = ReduceOut::kY);
 
