@@ -683,6 +683,8 @@ int tc_down_splits(const FwdShape &s, int num_sms) {
 }
 
 // Widest N tile from `cands` (descending) that still gives every SM a tile.
+constexpr bool kWideGateUpOneTile = true;
+
 static int pick_bn(int tiles_m, int n_total, std::initializer_list<int> cands, int num_sms) {
   int last = 0;
   for (int c : cands) {
@@ -759,8 +761,13 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
                              const float *sig, uint16_t *act, cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
   const int tiles_m = (int)((s.T + kBM - 1) / kBM);
-  // N tile: g and u of 128 channels (two banks) or of 64 channels (one bank)
-  const int bn = 2 * pick_bn(tiles_m, s.d_i, {128, 64}, dev.num_sms);
+  // N tile: g and u of 128 channels (two banks) or of 64 channels (one bank).
+  // One token tile: every N tile streams the whole x tile again, so the
+  // wider tile (half the x traffic per weight byte) wins even with fewer
+  // tiles than SMs.
+  const int bn = 2 * ((kWideGateUpOneTile && tiles_m == 1 && s.d_i % 128 == 0)
+                          ? 128
+                          : pick_bn(tiles_m, s.d_i, {128, 64}, dev.num_sms));
   CUtensorMap mX, mG, mU;
   if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mG, Wg, s.d, s.d_i, 64, bn / 2) ||
       !make_map(&mU, Wu, s.d, s.d_i, 64, bn / 2))
