@@ -52,6 +52,9 @@ def parse_args(argv=None):
                     choices=["decode", "batched_decode", "prefill", "long_prefill"])
     ap.add_argument("--impl", default="sfn", choices=["sfn", "reference"])
     ap.add_argument("--k", type=int, default=None, help="override top-k (e.g. 64: dense mask)")
+    ap.add_argument("--method", default="sfn", choices=["sfn", "dense4x"],
+                    help="sfn: the predictor-gated sparse FFN; dense4x: the pages' post-hoc "
+                         "comparison (dense gate/up, amplitude top-k, sparse down)")
     ap.add_argument("--path", default="auto", choices=["auto", "cuda_core", "tensor"],
                     help="kernels to use (the library picks by token count when auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -216,11 +219,17 @@ def stage_work(wl, T, union_channels):
                       "flops": 4 * T * d_s * d},
         "tc_down": {"bytes": union_channels * d * e + T * d_i * e + T * d * e,
                     "flops": 2 * T * d_s * d},
+        # Dense-4x: gate and up are dense (the mask depends on them)
+        "dense4x_gateup": {"bytes": 2 * d_i * d * e + T * d * e + T * d_i * e + T * nb * 8,
+                           "flops": 4 * T * d_i * d},
     }
 
 
-def useful_flops_per_token(wl):
-    """Predictor (2dr + 2r d_i) + kept gate and up (4 d d_s) + kept down (2 d d_s)."""
+def useful_flops_per_token(wl, method="sfn"):
+    """Predictor (2dr + 2r d_i) + kept gate and up (4 d d_s) + kept down (2 d d_s);
+    Dense-4x: dense gate and up (4 d d_i) + kept down (2 d d_s)."""
+    if method == "dense4x":
+        return 2 * (2 * wl.d * wl.d_i + wl.d * wl.d_s)
     return 2 * (wl.d * wl.r + wl.r * wl.d_i + 3 * wl.d * wl.d_s)
 
 
@@ -262,7 +271,11 @@ def run_sfn(args, rank, world, local):
     xs = [make_tokens_device(wl, dev, seed=rank, layer=i) for i in range(S)]
     ys = [torch.empty((T, wl.d), dtype=wl.torch_dtype, device=dev) for _ in range(S)]
     ms = [torch.empty((T, wl.n_banks), dtype=torch.int64, device=dev) for _ in range(S)]
-    ws_bytes = sfn.workspace_bytes(T, wl.d, wl.d_i, wl.r, wl.bank, wl.k, wl.torch_dtype)
+    dense4x = args.method == "dense4x"
+    if dense4x and wl.dtype != "bf16":
+        raise SystemExit("bench.py: the Dense-4x comparison runs on bf16 workloads")
+    ws_bytes = (L.sfn_dense4x_workspace_bytes(T, wl.d, wl.d_i, wl.bank, wl.k) if dense4x else
+                sfn.workspace_bytes(T, wl.d, wl.d_i, wl.r, wl.bank, wl.k, wl.torch_dtype))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     path_id = {"auto": 0, "cuda_core": 1, "tensor": 2}[args.path]
     stream = torch.cuda.Stream(device=dev)
@@ -272,7 +285,11 @@ def run_sfn(args, rank, world, local):
         ptrs = [xs[i].data_ptr(), lay["A"].data_ptr(), lay["B"].data_ptr(),
                 lay["Wg"].data_ptr(), lay["Wu"].data_ptr(), lay["Wd"].data_ptr(),
                 ys[i].data_ptr(), ms[i].data_ptr(), T, wl.d, wl.d_i, wl.r, wl.bank, wl.k]
-        if wl.dtype == "bf16":
+        if dense4x:
+            rc = L.sfn_dense4x_forward(ptrs[0], ptrs[3], ptrs[4], ptrs[5], ptrs[6], ptrs[7], T,
+                                       wl.d, wl.d_i, wl.bank, wl.k, ws.data_ptr(), ws_bytes,
+                                       st_ptr)
+        elif wl.dtype == "bf16":
             rc = L.sfn_sparse_ffn_forward_path(*ptrs, path_id, ws.data_ptr(), ws_bytes, st_ptr)
         else:
             rc = L.sfn_sparse_ffn_forward_f32_ws(*ptrs, ws.data_ptr(), ws_bytes, st_ptr)
@@ -408,9 +425,15 @@ def run_sfn(args, rank, world, local):
                 i = j % S
                 x_dev.copy_(x_host[i], non_blocking=True)
                 lay = layers[i]
-                sfn.sparse_ffn_forward(x_dev, lay["A"], lay["B"], lay["Wg"], lay["Wu"],
-                                       lay["Wd"], bank=wl.bank, k=wl.k, y=ys[i], mask=ms[i],
-                                       workspace=ws, path=args.path, stream=stream)
+                if dense4x:
+                    sfn.dense4x_forward(x_dev, lay["Wg"], lay["Wu"], lay["Wd"], bank=wl.bank,
+                                        k=wl.k, y=ys[i], mask=ms[i], workspace=ws,
+                                        stream=stream)
+                else:
+                    sfn.sparse_ffn_forward(x_dev, lay["A"], lay["B"], lay["Wg"], lay["Wu"],
+                                           lay["Wd"], bank=wl.bank, k=wl.k, y=ys[i],
+                                           mask=ms[i], workspace=ws, path=args.path,
+                                           stream=stream)
                 y_host.copy_(ys[i], non_blocking=True)
                 m_host.copy_(ms[i], non_blocking=True)
                 stream.synchronize()  # the caller reads the step's result
@@ -425,7 +448,8 @@ def run_sfn(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, {k: v.cpu() for k, v in layers[0].items()}, xs[0].cpu())
+        cpu = cpu_baseline(wl, {k: v.cpu() for k, v in layers[0].items()}, xs[0].cpu(),
+                           method=args.method)
 
     if world > 1:
         dist.barrier()
@@ -437,8 +461,9 @@ def run_sfn(args, rank, world, local):
 
     value = world * T * K / (elapsed_ms_max * 1e-3)
     # the path's algorithmic minimum: predictor weights, kept rows, x and y
-    step_bytes = sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "ffn", "reduce"))
-    step_flops = T * useful_flops_per_token(wl)
+    step_bytes = (sum(work[n]["bytes"] for n in ("dense4x_gateup", "tc_down")) if dense4x else
+                  sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "ffn", "reduce")))
+    step_flops = T * useful_flops_per_token(wl, args.method)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": elapsed_ms_max / K, "higher_is_better": True,
@@ -447,6 +472,7 @@ def run_sfn(args, rank, world, local):
             "workload": f"{wl.name}: T={T} d={wl.d} d_i={wl.d_i} r={wl.r} bank={wl.bank} "
                         f"k={wl.k} {wl.dtype}",
             "T": T, "d": wl.d, "d_i": wl.d_i, "r": wl.r, "bank": wl.bank, "k": wl.k,
+            "method": args.method,
             "l2": (f"inputs larger than L2: steps rotate over {S} distinct layers "
                    f"({S * sum(v.numel() * v.element_size() for v in layers[0].values()) / 1e9:.2f}"
                    " GB of weights)"),
@@ -477,26 +503,33 @@ def run_sfn(args, rank, world, local):
     return line
 
 
-def cpu_baseline(wl, layer_host, x_host, budget_s=12.0):
+def cpu_baseline(wl, layer_host, x_host, budget_s=12.0, method="sfn"):
     """The oracle, as it stands, on a bounded sample of the same workload."""
     import oracle
     oracle.build()
     cores = oracle.num_threads()
+
+    def run(xb):
+        if method == "dense4x":
+            oracle.dense4x(xb, layer_host["Wg"], layer_host["Wu"], layer_host["Wd"], wl.bank,
+                           wl.k)
+        else:
+            oracle.forward(xb, layer_host["A"], layer_host["B"], layer_host["Wg"],
+                           layer_host["Wu"], layer_host["Wd"], wl.bank, wl.k)
+
     t0 = time.perf_counter()
-    oracle.forward(x_host[:1], layer_host["A"], layer_host["B"], layer_host["Wg"],
-                   layer_host["Wu"], layer_host["Wd"], wl.bank, wl.k)
+    run(x_host[:1])
     t1 = time.perf_counter() - t0
     n = max(1, min(512, int(budget_s / max(t1, 1e-3)) * max(cores, 1) // 2))
     import torch
     reps = math.ceil(n / x_host.shape[0])
     xb = torch.cat([x_host] * reps)[:n]
     t0 = time.perf_counter()
-    oracle.forward(xb, layer_host["A"], layer_host["B"], layer_host["Wg"], layer_host["Wu"],
-                   layer_host["Wd"], wl.bank, wl.k)
+    run(xb)
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": UNIT, "cores": min(cores, n), "kind": "oracle",
             "sample": f"{n} tokens of the {wl.name} workload (T={wl.T} per step) through the "
-                      f"fp64 oracle, OpenMP over tokens, {dt:.1f} s"}
+                      f"fp64 oracle ({method}), OpenMP over tokens, {dt:.1f} s"}
 
 
 # ---------------------------------------------------------------- the reference arm
@@ -522,8 +555,11 @@ def run_reference(args, rank, world):
 
     def step(j):
         s = (j % 4) * T_step
-        oracle.forward(x[s:s + T_step], layer["A"], layer["B"], layer["Wg"], layer["Wu"],
-                       layer["Wd"], wl.bank, wl.k)
+        if args.method == "dense4x":
+            oracle.dense4x(x[s:s + T_step], layer["Wg"], layer["Wu"], layer["Wd"], wl.bank, wl.k)
+        else:
+            oracle.forward(x[s:s + T_step], layer["A"], layer["B"], layer["Wg"], layer["Wu"],
+                           layer["Wd"], wl.bank, wl.k)
 
     t0 = time.perf_counter()
     step(0)
@@ -544,7 +580,9 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} d_i={wl.d_i} r={wl.r} "
-                               f"bank={wl.bank} k={wl.k} {wl.dtype}"},
+                               f"bank={wl.bank} k={wl.k} {wl.dtype}",
+                   "T": wl.T, "d": wl.d, "d_i": wl.d_i, "r": wl.r, "bank": wl.bank, "k": wl.k,
+                   "method": args.method},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(cores, T_step),
                          "kind": "oracle",
                          "sample": f"{T_step} tokens per step (of T={wl.T}), {K_eff} steps"

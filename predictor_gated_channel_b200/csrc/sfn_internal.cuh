@@ -86,6 +86,8 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // channel i), identical in every lane.
 __device__ __forceinline__ uint64_t warp_bank_topk(uint32_t key0, uint32_t key1, int bank,
                                                    int k) {
+  // k = bank: the predictor-gated dense FFN (every channel kept), no ranking
+  if (k >= bank) return bank >= 64 ? ~0ull : ((1ull << bank) - 1ull);
   const int lane = threadIdx.x & 31;
   int r0 = 0, r1 = 0;
 #pragma unroll 8

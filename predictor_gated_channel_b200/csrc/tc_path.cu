@@ -198,6 +198,11 @@ __device__ __forceinline__ void keys_threshold(uint32_t (&s)[64], int k, uint32_
 // [taddr, taddr + 64) of this thread's row, and the number of keys strictly
 // above it.
 __device__ __forceinline__ void bank_threshold(uint32_t taddr, int k, uint32_t &tau, int &gt) {
+  if (k >= 64) {  // k = bank: every channel kept (key >= 0 = tau), no ranking
+    tau = 0u;
+    gt = 0;
+    return;
+  }
   uint32_t s[64];
   tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
   tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
