@@ -63,6 +63,9 @@ def _open(path: str):
         vp, vp, vp]
     lib.sfn_oracle_dense_then_mask.argtypes = [
         vp, ci, vp, vp, vp, ci, vp, ci, vp, ci, i64, ci, ci, ci, vp]
+    lib.sfn_oracle_backward.argtypes = [vp, ci, vp, ci, vp, ci, vp, ci, vp, ci, vp, ci, vp, ci,
+                                        i64, ci, ci, ci, ci, ci, ctypes.c_double, vp, vp, vp,
+                                        vp, vp, vp, vp, vp]
     lib.sfn_oracle_num_threads.restype = ci
     lib.sfn_oracle_dense4x.argtypes = [vp, ci, vp, ci, vp, ci, vp, ci, i64, ci, ci, ci, ci, ci,
                                        vp, vp, vp]
@@ -222,3 +225,43 @@ def mask_to_bool(mask, bank: int) -> np.ndarray:
     m = np.asarray(mask, dtype=np.uint64)
     bits = (m[..., None] >> np.arange(bank, dtype=np.uint64)) & np.uint64(1)
     return bits.reshape(m.shape[0], -1).astype(bool)
+
+
+def backward(x, A, B, Wg, Wu, Wd, dy, bank: int, k: int, temp: float, mask=None) -> dict:
+    """Gradients of L = sum(dy * y) through the whole layer, with the soft
+    surrogate gradient of the hard top-k (threshold tau_b = midpoint of the
+    bank's k-th and (k+1)-th logits, held constant; dm/dp := sigma'((p -
+    tau_b) / temp) / temp).  Returns float64 arrays dx [T, d], dA [r, d],
+    dB [d_i, r], dWg, dWu, dWd [d_i, d] and the mask used (uint64 [T, d_i /
+    bank]).  With ``mask`` given, that mask replaces the own top-k."""
+    xa, xd = _arr(x)
+    Aa, Ad = _arr(A)
+    Ba, Bd = _arr(B)
+    ga, gd = _arr(Wg)
+    ua, ud = _arr(Wu)
+    wa, wd = _arr(Wd)
+    ya, yd = _arr(dy)
+    T, d = xa.shape
+    r = Aa.shape[0]
+    d_i = Ba.shape[0]
+    assert Aa.shape == (r, d) and Ba.shape == (d_i, r) and ya.shape == (T, d)
+    assert ga.shape == ua.shape == wa.shape == (d_i, d)
+    assert d_i % bank == 0 and 1 <= k <= bank <= 64 and temp > 0
+    nb = d_i // bank
+    out = {"dx": np.empty((T, d)), "dA": np.empty((r, d)), "dB": np.empty((d_i, r)),
+           "dWg": np.empty((d_i, d)), "dWu": np.empty((d_i, d)), "dWd": np.empty((d_i, d)),
+           "mask": np.empty((T, nb), np.uint64)}
+    m_in = None
+    if mask is not None:
+        if hasattr(mask, "detach"):
+            mask = mask.detach().cpu().numpy()
+        m_in = np.ascontiguousarray(np.asarray(mask))
+        m_in = m_in.view(np.uint64) if m_in.dtype == np.int64 else m_in.astype(np.uint64)
+        assert m_in.shape == (T, nb)
+    _load().sfn_oracle_backward(_ptr(xa), xd, _ptr(Aa), Ad, _ptr(Ba), Bd, _ptr(ga), gd, _ptr(ua),
+                                ud, _ptr(wa), wd, _ptr(ya), yd, T, d, d_i, r, bank, k,
+                                float(temp), None if m_in is None else _ptr(m_in),
+                                _ptr(out["dx"]), _ptr(out["dA"]), _ptr(out["dB"]),
+                                _ptr(out["dWg"]), _ptr(out["dWu"]), _ptr(out["dWd"]),
+                                _ptr(out["mask"]))
+    return out

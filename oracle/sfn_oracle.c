@@ -246,6 +246,142 @@ void sfn_oracle_dense4x(const void *x, int x_dt, const void *Wg, int Wg_dt, cons
 }
 
 /* Threads the OpenMP runtime will use (reported beside CPU timings). */
+/* Backward of the whole layer, for predictor training ("Executie / Backward
+ * Pass" in the architecture section of the same summary: the hard top-k is
+ * not differentiable, so a soft, sigmoid-like surrogate gradient around the
+ * selection threshold lets the loss reach the predictor).
+ *
+ * The forward is the one above: h = A x, p = B h, m_j = hard bank top-k,
+ * s_j = sigma(p_j), g_j = Wg[j].x, u_j = Wu[j].x, a_j = m_j s_j g_j u_j,
+ * y = sum_j a_j Wd[j].  Given dy = dL/dy this returns dL/dx, dL/dA, dL/dB,
+ * dL/dWg, dL/dWu, dL/dWd, with one reading for the surrogate (the pages
+ * give neither formula nor temperature):
+ *   - bank b's threshold is tau_b = (p_(k) + p_(k+1)) / 2, the midpoint of
+ *     its k-th and (k+1)-th logits in the ranking order; it is held constant
+ *     (no gradient flows through it).  With k = bank there is no threshold
+ *     and no surrogate term;
+ *   - dm_j/dp_j is replaced by sigma'(z_j) / temp with z_j = (p_j - tau_b) /
+ *     temp and sigma'(z) = sigma(z) (1 - sigma(z)): the derivative of a
+ *     sigmoid step of width temp centred on the threshold.  m_j itself stays
+ *     hard (0 or 1) everywhere else.
+ * The chain rule then gives, per token and channel j (da_j = Wd[j].dy):
+ *   dg_j = da_j m_j s_j u_j,   du_j = da_j m_j s_j g_j,
+ *   dp_j = da_j g_j u_j (m_j s_j (1 - s_j) + s_j sigma'(z_j) / temp),
+ *   dWd[j] += a_j dy,  dWg[j] += dg_j x,  dWu[j] += du_j x,  dB[j] += dp_j h,
+ *   dh = sum_j dp_j B[j],  dA += dh x^T,
+ *   dx = sum_j (dg_j Wg[j] + du_j Wu[j]) + A^T dh.
+ * The surrogate term needs g_j u_j of every channel, kept or not.
+ *
+ * mask_in (may be NULL): use this mask instead of the own top-k (the
+ * threshold still comes from the own logits).  mask_out (may be NULL)
+ * receives the mask used.  Every gradient output is overwritten. */
+void sfn_oracle_backward(const void *x, int x_dt, const void *A, int A_dt,
+                         const void *B, int B_dt, const void *Wg, int Wg_dt,
+                         const void *Wu, int Wu_dt, const void *Wd, int Wd_dt,
+                         const void *dy, int dy_dt, int64_t T, int d, int d_i,
+                         int r, int bank, int k, double temp,
+                         const uint64_t *mask_in, double *dx, double *dA,
+                         double *dB, double *dWg, double *dWu, double *dWd,
+                         uint64_t *mask_out) {
+  const int nb = d_i / bank;
+  memset(dA, 0, sizeof(double) * (size_t)r * d);
+  memset(dB, 0, sizeof(double) * (size_t)d_i * r);
+  memset(dWg, 0, sizeof(double) * (size_t)d_i * d);
+  memset(dWu, 0, sizeof(double) * (size_t)d_i * d);
+  memset(dWd, 0, sizeof(double) * (size_t)d_i * d);
+  double *h = (double *)malloc(sizeof(double) * (size_t)r);
+  double *dh = (double *)malloc(sizeof(double) * (size_t)r);
+  double *p = (double *)malloc(sizeof(double) * (size_t)d_i);
+  double *tau = (double *)malloc(sizeof(double) * (size_t)nb);
+  double *dg = (double *)malloc(sizeof(double) * (size_t)d_i);
+  double *du = (double *)malloc(sizeof(double) * (size_t)d_i);
+  uint64_t *mw = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)nb);
+  for (int64_t t = 0; t < T; ++t) {
+    /* forward of this token: h, p, mask, thresholds */
+    for (int m = 0; m < r; ++m) {
+      double acc = 0.0;
+      for (int n = 0; n < d; ++n) acc += ld(x, x_dt, t * d + n) * ld(A, A_dt, (int64_t)m * d + n);
+      h[m] = acc;
+    }
+    for (int j = 0; j < d_i; ++j) {
+      double acc = 0.0;
+      for (int m = 0; m < r; ++m) acc += h[m] * ld(B, B_dt, m + (int64_t)j * r);
+      p[j] = acc;
+    }
+    for (int b = 0; b < nb; ++b) {
+      const double *pb = p + (int64_t)b * bank;
+      uint64_t word = 0;
+      double pk = 0.0, pk1 = 0.0;
+      for (int j = 0; j < bank; ++j) {
+        int rk = 0;
+        for (int i = 0; i < bank; ++i)
+          if (beats(pb[i], pb[j]) || (same(pb[i], pb[j]) && i < j)) ++rk;
+        if (rk < k) word |= ((uint64_t)1) << j;
+        if (rk == k - 1) pk = pb[j];
+        if (rk == k) pk1 = pb[j];
+      }
+      tau[b] = (k < bank) ? 0.5 * (pk + pk1) : NAN;
+      mw[b] = mask_in ? mask_in[t * nb + b] : word;
+      if (mask_out) mask_out[t * nb + b] = mw[b];
+    }
+    /* every channel: g, u, da; the chain rule; weight gradients of row j */
+#pragma omp parallel for schedule(static)
+    for (int j = 0; j < d_i; ++j) {
+      double g = 0.0, u = 0.0, da = 0.0;
+      for (int n = 0; n < d; ++n) {
+        const double xn = ld(x, x_dt, t * d + n);
+        g += ld(Wg, Wg_dt, (int64_t)j * d + n) * xn;
+        u += ld(Wu, Wu_dt, (int64_t)j * d + n) * xn;
+        da += ld(Wd, Wd_dt, (int64_t)j * d + n) * ld(dy, dy_dt, t * d + n);
+      }
+      const double mj = (double)((mw[j / bank] >> (j % bank)) & 1);
+      const double s = sfn_oracle_sigmoid(p[j]);
+      const double tb = tau[j / bank];
+      double sur = 0.0;
+      if (!isnan(tb)) {
+        const double sz = sfn_oracle_sigmoid((p[j] - tb) / temp);
+        sur = sz * (1.0 - sz) / temp;
+      }
+      const double a = mj * s * g * u;
+      dg[j] = da * mj * s * u;
+      du[j] = da * mj * s * g;
+      const double dp = da * g * u * (mj * s * (1.0 - s) + s * sur);
+      for (int n = 0; n < d; ++n) {
+        const double xn = ld(x, x_dt, t * d + n);
+        dWd[(int64_t)j * d + n] += a * ld(dy, dy_dt, t * d + n);
+        dWg[(int64_t)j * d + n] += dg[j] * xn;
+        dWu[(int64_t)j * d + n] += du[j] * xn;
+      }
+      for (int m = 0; m < r; ++m) dB[(int64_t)j * r + m] += dp * h[m];
+      p[j] = dp; /* p[j] is not read again for this token: keep dp there */
+    }
+    /* dh = B^T dp (p now holds dp), dA += dh x^T */
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < r; ++m) {
+      double acc = 0.0;
+      for (int j = 0; j < d_i; ++j) acc += p[j] * ld(B, B_dt, m + (int64_t)j * r);
+      dh[m] = acc;
+      for (int n = 0; n < d; ++n) dA[(int64_t)m * d + n] += acc * ld(x, x_dt, t * d + n);
+    }
+    /* dx = Wg^T dg + Wu^T du + A^T dh */
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < d; ++n) {
+      double acc = 0.0;
+      for (int j = 0; j < d_i; ++j)
+        acc += dg[j] * ld(Wg, Wg_dt, (int64_t)j * d + n) + du[j] * ld(Wu, Wu_dt, (int64_t)j * d + n);
+      for (int m = 0; m < r; ++m) acc += dh[m] * ld(A, A_dt, (int64_t)m * d + n);
+      dx[t * d + n] = acc;
+    }
+  }
+  free(h);
+  free(dh);
+  free(p);
+  free(tau);
+  free(dg);
+  free(du);
+  free(mw);
+}
+
 int sfn_oracle_num_threads(void) {
 #ifdef _OPENMP
   extern int omp_get_max_threads(void);

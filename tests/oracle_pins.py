@@ -263,9 +263,117 @@ def pin_dense4x():
         assert np.allclose(y, ((Wd.T) @ (keep * act).T).T, rtol=1e-11, atol=1e-12)
 
 
+# ------------------------------------------------------------------ backward
+# Reading pinned here ("Executie / Backward Pass" of the same architecture
+# section: a sigmoid-like surrogate gradient around the selection threshold):
+# tau_b = midpoint of bank b's k-th and (k+1)-th logits, held constant;
+# dm_j/dp_j := sigma'((p_j - tau_b) / temp) / temp; the forward mask stays hard.
+
+def _surrogate_grads_torch(x, A, B, Wg, Wu, Wd, dy, bank, k, temp):
+    """Gradients by float64 autograd of a straight-through forward whose value
+    is the hard-masked layer and whose mask derivative is the surrogate; the
+    chain rule is torch's, not the oracle's."""
+    import torch
+    ts = [torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (x, A, B, Wg, Wu, Wd)]
+    tx, tA, tB, tg, tu, td = ts
+    p = (tx @ tA.T) @ tB.T
+    T, d_i = p.shape
+    pb = p.view(T, d_i // bank, bank)
+    order = torch.from_numpy(np.argsort(-pb.detach().numpy(), axis=2, kind="stable"))
+    hard = torch.zeros_like(pb).scatter_(2, order[:, :, :k], 1.0)
+    if k < bank:
+        vals = torch.gather(pb.detach(), 2, order)
+        tau = 0.5 * (vals[:, :, k - 1] + vals[:, :, k])
+        soft = torch.sigmoid((pb - tau[:, :, None]) / temp)
+        m = hard + soft - soft.detach()
+    else:
+        m = hard
+    a = m.reshape(T, d_i) * torch.sigmoid(p) * (tx @ tg.T) * (tx @ tu.T)
+    loss = ((a @ td) * torch.tensor(dy, dtype=torch.float64)).sum()
+    grads = torch.autograd.grad(loss, ts)
+    return dict(zip(["dx", "dA", "dB", "dWg", "dWu", "dWd"], [g.numpy() for g in grads]))
+
+
+def pin_backward_autograd():
+    """Oracle backward = float64 autograd of the straight-through surrogate
+    forward (several bank / k / temperature cases, k = bank included)."""
+    for seed, (d, d_i, r, bank, k, temp) in enumerate(
+            [(12, 32, 6, 8, 3, 0.3), (20, 64, 5, 16, 4, 2.0), (9, 24, 4, 8, 8, 0.5),
+             (16, 128, 8, 64, 16, 0.1)]):
+        rng = _rng(100 + seed)
+        x, A, B, Wg, Wu, Wd = _layer(rng, d, d_i, r, scale=2.0)
+        dy = rng.standard_normal(x.shape)
+        ref = _surrogate_grads_torch(x, A, B, Wg, Wu, Wd, dy, bank, k, temp)
+        got = oracle.backward(x, A, B, Wg, Wu, Wd, dy, bank, k, temp)
+        for name, v in ref.items():
+            assert np.allclose(got[name], v, rtol=1e-9, atol=1e-12), (name, bank, k)
+
+
+def pin_backward_finite_differences():
+    """With a vanishing temperature the surrogate is zero away from the
+    threshold, so the backward must equal central differences of
+    L = sum(dy * y) through the oracle's own forward (mask unchanged by the
+    perturbation)."""
+    rng = _rng(7)
+    bank, k, temp, eps = 8, 3, 1e-9, 1e-6
+    x, A, B, Wg, Wu, Wd = _layer(rng, 10, 32, 5, scale=2.0)
+    dy = rng.standard_normal(x.shape)
+    ins = {"dx": x, "dA": A, "dB": B, "dWg": Wg, "dWu": Wu, "dWd": Wd}
+    order = ["dx", "dA", "dB", "dWg", "dWu", "dWd"]
+    got = oracle.backward(x, A, B, Wg, Wu, Wd, dy, bank, k, temp)
+    _, _, m0 = oracle.forward(x, A, B, Wg, Wu, Wd, bank=bank, k=k)
+
+    def loss(args):
+        y, _, m = oracle.forward(*args, bank=bank, k=k)
+        assert np.array_equal(m, m0), "perturbation flipped the mask"
+        return float((y * dy).sum())
+
+    for name in order:
+        arr = ins[name]
+        for idx in [tuple(rng.integers(0, s) for s in arr.shape) for _ in range(5)]:
+            args_p = [ins[n].copy() for n in order]
+            args_m = [ins[n].copy() for n in order]
+            args_p[order.index(name)][idx] += eps
+            args_m[order.index(name)][idx] -= eps
+            fd = (loss(args_p) - loss(args_m)) / (2 * eps)
+            assert abs(fd - got[name][idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd,
+                                                                        got[name][idx])
+
+
+def pin_backward_closed_form():
+    """A one-token layer worked by hand: d = r = 1, two channels in one bank,
+    k = 1.  x = 1, A = 1, B = (2, 1) -> h = 1, p = (2, 1): channel 0 kept,
+    channel 1 not, tau = 1.5.  g = (0.5, 1.5), u = (2, -1), dy = 1, Wd = (1, 3)
+    -> da = (1, 3).  With s_j = sigma(p_j), z_j = (p_j - 1.5) / temp and
+    q_j = sigma(z_j)(1 - sigma(z_j)) / temp:
+      dp_0 = g0 u0 (s0 (1 - s0) + s0 q0),   dp_1 = 3 g1 u1 s1 q1 (surrogate only),
+      dWd = (s0 g0 u0, 0), dWg = (s0 u0, 0), dWu = (s0 g0, 0), dB = (dp_0, dp_1),
+      dh = 2 dp_0 + dp_1 = dA,  dx = s0 u0 0.5 + s0 g0 2 + dh."""
+    sg = lambda z: 1.0 / (1.0 + math.exp(-z))
+    for temp in (0.25, 1.0, 3.0):
+        x = np.array([[1.0]]); A = np.array([[1.0]]); B = np.array([[2.0], [1.0]])
+        Wg = np.array([[0.5], [1.5]]); Wu = np.array([[2.0], [-1.0]]); Wd = np.array([[1.0], [3.0]])
+        dy = np.array([[1.0]])
+        g0, g1, u0, u1 = 0.5, 1.5, 2.0, -1.0
+        s0, s1 = sg(2.0), sg(1.0)
+        q0 = sg(0.5 / temp) * (1 - sg(0.5 / temp)) / temp
+        q1 = sg(-0.5 / temp) * (1 - sg(-0.5 / temp)) / temp
+        dp0 = g0 * u0 * (s0 * (1 - s0) + s0 * q0)
+        dp1 = 3.0 * g1 * u1 * s1 * q1
+        dh = 2 * dp0 + dp1
+        want = {"dWd": [[s0 * g0 * u0], [0.0]], "dWg": [[s0 * u0], [0.0]],
+                "dWu": [[s0 * g0], [0.0]], "dB": [[dp0], [dp1]], "dA": [[dh]],
+                "dx": [[s0 * u0 * 0.5 + s0 * g0 * 2.0 + dh]]}
+        got = oracle.backward(x, A, B, Wg, Wu, Wd, dy, bank=2, k=1, temp=temp)
+        assert int(got["mask"][0, 0]) == 1
+        for name, v in want.items():
+            assert np.allclose(got[name], np.array(v), rtol=1e-12, atol=1e-15), (name, temp)
+
+
 ALL_PINS = [
     pin_topk_golden, pin_topk_popcount, pin_topk_stable_sort, pin_topk_brute_force,
     pin_predict_matmul, pin_predict_selector, pin_predict_integer_exact, pin_sigmoid,
     pin_forward_golden, pin_forward_k_equals_bank, pin_forward_masked_dense,
     pin_forward_invariants, pin_forward_bf16_widening, pin_dense4x,
+    pin_backward_autograd, pin_backward_finite_differences, pin_backward_closed_form,
 ]

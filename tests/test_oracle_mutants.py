@@ -35,6 +35,16 @@ MUTANTS = {
     "dense4x_amplitude_signed": ("amp[j] = fabs(act[j]);", "amp[j] = act[j];"),
     "dense4x_gate_not_silu": ("act[j] = g * sfn_oracle_sigmoid(g) * u;",
                               "act[j] = sfn_oracle_sigmoid(g) * u;"),
+    "bwd_surrogate_dropped": ("(mj * s * (1.0 - s) + s * sur)", "(mj * s * (1.0 - s))"),
+    "bwd_surrogate_unscaled": ("sur = sz * (1.0 - sz) / temp;", "sur = sz * (1.0 - sz);"),
+    "bwd_threshold_is_kth": ("tau[b] = (k < bank) ? 0.5 * (pk + pk1) : NAN;",
+                             "tau[b] = (k < bank) ? pk : NAN;"),
+    "bwd_du_uses_u": ("du[j] = da * mj * s * g;", "du[j] = da * mj * s * u;"),
+    "bwd_sigmoid_derivative_dropped": ("(mj * s * (1.0 - s) + s * sur)", "(mj * s + s * sur)"),
+    "bwd_dx_without_predictor": ("for (int m = 0; m < r; ++m) acc += dh[m] * ld(A",
+                                 "for (int m = 0; m < 0; ++m) acc += dh[m] * ld(A"),
+    "bwd_dA_without_x": ("dA[(int64_t)m * d + n] += acc * ld(x, x_dt, t * d + n);",
+                         "dA[(int64_t)m * d + n] += acc;"),
 }
 
 
