@@ -52,9 +52,12 @@ def parse_args(argv=None):
                     choices=["decode", "batched_decode", "prefill", "long_prefill"])
     ap.add_argument("--impl", default="sfn", choices=["sfn", "reference"])
     ap.add_argument("--k", type=int, default=None, help="override top-k (e.g. 64: dense mask)")
-    ap.add_argument("--method", default="sfn", choices=["sfn", "dense4x"],
+    ap.add_argument("--method", default="sfn", choices=["sfn", "dense4x", "backward"],
                     help="sfn: the predictor-gated sparse FFN; dense4x: the pages' post-hoc "
-                         "comparison (dense gate/up, amplitude top-k, sparse down)")
+                         "comparison (dense gate/up, amplitude top-k, sparse down); backward: "
+                         "the layer's backward with the surrogate top-k gradient")
+    ap.add_argument("--temperature", type=float, default=1.0,
+                    help="surrogate temperature of --method backward")
     ap.add_argument("--path", default="auto", choices=["auto", "cuda_core", "tensor"],
                     help="kernels to use (the library picks by token count when auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -222,6 +225,13 @@ def stage_work(wl, T, union_channels):
         # Dense-4x: gate and up are dense (the mask depends on them)
         "dense4x_gateup": {"bytes": 2 * d_i * d * e + T * d * e + T * d_i * e + T * nb * 8,
                            "flops": 4 * T * d_i * d},
+        # backward: g, u, da; dWd, dWg, dWu; dx (two d_i contractions) are 8
+        # T d d_i GEMMs, plus dh, dB (T d_i r each) and dA, dx (T r d each)
+        "bwd_gemm": {"bytes": 5 * d_i * d * e + 3 * d_i * d * 4 + 2 * d_i * r * e
+                              + T * d_i * (3 * 4 + 4 * e) + 2 * T * d * e + T * d * 4,
+                     "flops": 2 * T * (8 * d * d_i + 2 * d_i * r + 2 * r * d)},
+        "bwd_elem": {"bytes": T * d_i * (4 * 4 + 4 * e) + T * nb * 12, "flops": 0},
+        "bwd_tau": {"bytes": T * d_i * 4 + T * nb * 12, "flops": 0},
     }
 
 
@@ -230,6 +240,9 @@ def useful_flops_per_token(wl, method="sfn"):
     Dense-4x: dense gate and up (4 d d_i) + kept down (2 d d_s)."""
     if method == "dense4x":
         return 2 * (2 * wl.d * wl.d_i + wl.d * wl.d_s)
+    if method == "backward":  # predictor recompute + the backward's contractions
+        return 2 * (wl.d * wl.r + wl.r * wl.d_i + 8 * wl.d * wl.d_i + 2 * wl.d_i * wl.r
+                    + 2 * wl.r * wl.d)
     return 2 * (wl.d * wl.r + wl.r * wl.d_i + 3 * wl.d * wl.d_s)
 
 
@@ -272,10 +285,22 @@ def run_sfn(args, rank, world, local):
     ys = [torch.empty((T, wl.d), dtype=wl.torch_dtype, device=dev) for _ in range(S)]
     ms = [torch.empty((T, wl.n_banks), dtype=torch.int64, device=dev) for _ in range(S)]
     dense4x = args.method == "dense4x"
-    if dense4x and wl.dtype != "bf16":
-        raise SystemExit("bench.py: the Dense-4x comparison runs on bf16 workloads")
-    ws_bytes = (L.sfn_dense4x_workspace_bytes(T, wl.d, wl.d_i, wl.bank, wl.k) if dense4x else
-                sfn.workspace_bytes(T, wl.d, wl.d_i, wl.r, wl.bank, wl.k, wl.torch_dtype))
+    backward = args.method == "backward"
+    if (dense4x or backward) and wl.dtype != "bf16":
+        raise SystemExit(f"bench.py: --method {args.method} runs on bf16 workloads")
+    if dense4x:
+        ws_bytes = L.sfn_dense4x_workspace_bytes(T, wl.d, wl.d_i, wl.bank, wl.k)
+    elif backward:
+        ws_bytes = L.sfn_backward_workspace_bytes(T, wl.d, wl.d_i, wl.r, wl.bank, wl.k)
+        # dy per rotation layer; one set of float32 gradients, overwritten every step
+        gen = torch.Generator(device=dev).manual_seed(1000 + rank)
+        dys = [torch.randn((T, wl.d), device=dev, generator=gen).to(torch.bfloat16)
+               for _ in range(S)]
+        gshape = {"dx": (T, wl.d), "dA": (wl.r, wl.d), "dB": (wl.d_i, wl.r),
+                  "dWg": (wl.d_i, wl.d), "dWu": (wl.d_i, wl.d), "dWd": (wl.d_i, wl.d)}
+        grads = {n: torch.empty(sh, dtype=torch.float32, device=dev) for n, sh in gshape.items()}
+    else:
+        ws_bytes = sfn.workspace_bytes(T, wl.d, wl.d_i, wl.r, wl.bank, wl.k, wl.torch_dtype)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     path_id = {"auto": 0, "cuda_core": 1, "tensor": 2}[args.path]
     stream = torch.cuda.Stream(device=dev)
@@ -285,7 +310,12 @@ def run_sfn(args, rank, world, local):
         ptrs = [xs[i].data_ptr(), lay["A"].data_ptr(), lay["B"].data_ptr(),
                 lay["Wg"].data_ptr(), lay["Wu"].data_ptr(), lay["Wd"].data_ptr(),
                 ys[i].data_ptr(), ms[i].data_ptr(), T, wl.d, wl.d_i, wl.r, wl.bank, wl.k]
-        if dense4x:
+        if backward:
+            gp = [grads[n].data_ptr() for n in ("dx", "dA", "dB", "dWg", "dWu", "dWd")]
+            rc = L.sfn_sparse_ffn_backward(*ptrs[:6], dys[i].data_ptr(), args.temperature, *gp,
+                                           ptrs[7], T, wl.d, wl.d_i, wl.r, wl.bank, wl.k,
+                                           ws.data_ptr(), ws_bytes, st_ptr)
+        elif dense4x:
             rc = L.sfn_dense4x_forward(ptrs[0], ptrs[3], ptrs[4], ptrs[5], ptrs[6], ptrs[7], T,
                                        wl.d, wl.d_i, wl.bank, wl.k, ws.data_ptr(), ws_bytes,
                                        st_ptr)
@@ -383,7 +413,10 @@ def run_sfn(args, rank, world, local):
         if n_arr[s_id]:
             name = L.sfn_stage_name(s_id).decode()
             stages[name] = {"launches": int(n_arr[s_id]), "ms_total": ms_arr[s_id],
-                            "us_per_launch": 1e3 * ms_arr[s_id] / n_arr[s_id]}
+                            "us_per_launch": 1e3 * ms_arr[s_id] / n_arr[s_id],
+                            # a stage may run more than once per step (split-K sums,
+                            # the backward's groups of GEMMs): work is per step
+                            "us_per_step": 1e3 * ms_arr[s_id] / n_stage_steps}
     tot = sum(v["ms_total"] for v in stages.values()) or 1.0
     for v in stages.values():
         v["share"] = v["ms_total"] / tot
@@ -392,7 +425,7 @@ def run_sfn(args, rank, world, local):
     if "tc_down" in stages and "reduce" in stages:  # split-K partial sums
         work["reduce"] = {"bytes": T * wl.d * 4, "flops": 0}
     dom = max(stages, key=lambda n: stages[n]["ms_total"])
-    dom_s = stages[dom]["us_per_launch"] * 1e-6
+    dom_s = stages[dom]["us_per_step"] * 1e-6
     if bound == "hbm":
         achieved = work[dom]["bytes"] / dom_s / 1e9
         peak, unit = peaks["hbm_gbs"], "GB/s"
@@ -404,11 +437,11 @@ def run_sfn(args, rank, world, local):
     traffic = traffic_from_profiles(dom, args.workload)
     for n, v in stages.items():
         v["alg_bytes_per_launch"] = work[n]["bytes"]
-        v["alg_gbs"] = work[n]["bytes"] / (v["us_per_launch"] * 1e-6) / 1e9
+        v["alg_gbs"] = work[n]["bytes"] / (v["us_per_step"] * 1e-6) / 1e9
 
     # end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not backward:
         n_e2e = min(K, 300 if T <= 64 else 10)
         x_host = [xs[i].cpu().pin_memory() for i in range(S)]
         y_host = torch.empty((T, wl.d), dtype=wl.torch_dtype).pin_memory()
@@ -461,8 +494,13 @@ def run_sfn(args, rank, world, local):
 
     value = world * T * K / (elapsed_ms_max * 1e-3)
     # the path's algorithmic minimum: predictor weights, kept rows, x and y
-    step_bytes = (sum(work[n]["bytes"] for n in ("dense4x_gateup", "tc_down")) if dense4x else
-                  sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "ffn", "reduce")))
+    if dense4x:
+        step_bytes = sum(work[n]["bytes"] for n in ("dense4x_gateup", "tc_down"))
+    elif backward:
+        step_bytes = sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "bwd_gemm",
+                                                    "bwd_elem", "bwd_tau"))
+    else:
+        step_bytes = sum(work[n]["bytes"] for n in ("pred_h", "logits_topk", "ffn", "reduce"))
     step_flops = T * useful_flops_per_token(wl, args.method)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -505,6 +543,8 @@ def run_sfn(args, rank, world, local):
 
 def cpu_baseline(wl, layer_host, x_host, budget_s=12.0, method="sfn"):
     """The oracle, as it stands, on a bounded sample of the same workload."""
+    import numpy as np
+
     import oracle
     oracle.build()
     cores = oracle.num_threads()
@@ -513,6 +553,10 @@ def cpu_baseline(wl, layer_host, x_host, budget_s=12.0, method="sfn"):
         if method == "dense4x":
             oracle.dense4x(xb, layer_host["Wg"], layer_host["Wu"], layer_host["Wd"], wl.bank,
                            wl.k)
+        elif method == "backward":
+            dy = np.random.default_rng(1000).standard_normal(xb.shape)
+            oracle.backward(xb, layer_host["A"], layer_host["B"], layer_host["Wg"],
+                            layer_host["Wu"], layer_host["Wd"], dy, wl.bank, wl.k, 1.0)
         else:
             oracle.forward(xb, layer_host["A"], layer_host["B"], layer_host["Wg"],
                            layer_host["Wu"], layer_host["Wd"], wl.bank, wl.k)
@@ -537,6 +581,7 @@ def cpu_baseline(wl, layer_host, x_host, budget_s=12.0, method="sfn"):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
+    import numpy as np
     import torch
 
     import oracle
@@ -557,6 +602,10 @@ def run_reference(args, rank, world):
         s = (j % 4) * T_step
         if args.method == "dense4x":
             oracle.dense4x(x[s:s + T_step], layer["Wg"], layer["Wu"], layer["Wd"], wl.bank, wl.k)
+        elif args.method == "backward":
+            dy = np.random.default_rng(1000 + j).standard_normal((T_step, wl.d))
+            oracle.backward(x[s:s + T_step], layer["A"], layer["B"], layer["Wg"], layer["Wu"],
+                            layer["Wd"], dy, wl.bank, wl.k, args.temperature)
         else:
             oracle.forward(x[s:s + T_step], layer["A"], layer["B"], layer["Wg"], layer["Wu"],
                            layer["Wd"], wl.bank, wl.k)

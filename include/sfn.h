@@ -239,6 +239,43 @@ sfn_status sfn_dense4x_forward(const void *x, const void *Wg, const void *Wu, co
                                int k, void *workspace, size_t workspace_bytes,
                                sfn_stream_t stream);
 
+/*
+ * Backward of the layer, for training the predictor ("1. Architectuur",
+ * Executie / Backward Pass: the non-differentiable top-k gets a soft,
+ * sigmoid-like surrogate gradient around the selection threshold).
+ *
+ * Given dy = dL/dy [T][d] for the forward above on the same inputs, writes
+ * the gradients of L with respect to every input:
+ *   dx [T][d], dA [r][d], dB [d_i][r], dWg, dWu, dWd [d_i][d]  (float32)
+ * Any of them may be NULL (not computed).  They are overwritten, not
+ * accumulated.  mask (may be NULL) receives the forward's mask [T][d_i/bank].
+ *
+ * Surrogate (a reading; the pages give no formula): bank b's threshold
+ * tau_b = (p_(k) + p_(k+1)) / 2, the midpoint of its k-th and (k+1)-th
+ * logits, held constant; the forward mask m stays hard; in the backward
+ * dm_j/dp_j := sigma'((p_j - tau_b) / temperature) / temperature.  With
+ * k = bank there is no threshold and no surrogate term.  The surrogate term
+ * needs g_j u_j of every channel, so the backward is dense in gate and up.
+ *
+ * bf16 inputs (x, A, B, Wg, Wu, Wd, dy); logits are recomputed with the
+ * forward's own kernels (the same mask as the forward for the same T), the
+ * elementwise chain rule runs in this library's kernels, and the dense
+ * contractions use cuBLAS (bf16 operands, float32 accumulation), loaded at
+ * run time: SFN_ERR_UNSUPPORTED if libcublas.so.12 cannot be loaded.
+ * temperature must be finite and > 0 (else SFN_ERR_INVALID_VALUE); d_i must
+ * be a multiple of 4.  Scratch: at least sfn_backward_workspace_bytes()
+ * bytes, 256-byte aligned (1.4 GB for 4096 tokens of the 4096 x 14336
+ * layer).  Other errors as sfn_sparse_ffn_forward_ws.
+ */
+size_t sfn_backward_workspace_bytes(int64_t T, int d, int d_i, int r, int bank, int k);
+sfn_status sfn_sparse_ffn_backward(const void *x, const void *A, const void *B, const void *Wg,
+                                   const void *Wu, const void *Wd, const void *dy,
+                                   float temperature, float *dx, float *dA, float *dB,
+                                   float *dWg, float *dWu, float *dWd, uint64_t *mask,
+                                   int64_t T, int d, int d_i, int r, int bank, int k,
+                                   void *workspace, size_t workspace_bytes,
+                                   sfn_stream_t stream);
+
 /* float32 twins of the two forward entry points. */
 sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
                                       const float *Wg, const float *Wu, const float *Wd,
@@ -271,6 +308,9 @@ enum {
   SFN_STAGE_TC_GATEUP = 7,    /* tensor cores: masked sigma(p) g u      */
   SFN_STAGE_TC_DOWN = 8,      /* tensor cores: y = act W_down           */
   SFN_STAGE_DENSE4X_GATEUP = 10, /* Dense-4x: silu(g) u + amplitude top-k */
+  SFN_STAGE_BWD_TAU = 11,     /* backward: mask and thresholds          */
+  SFN_STAGE_BWD_ELEM = 12,    /* backward: surrogate chain rule         */
+  SFN_STAGE_BWD_GEMM = 13,    /* backward: cuBLAS contractions          */
   SFN_STAGE_COUNT = 16        /* room for the stage ids of this library */
 };
 sfn_status sfn_timing_begin(void);

@@ -185,3 +185,39 @@ def dense4x_forward(x, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None, mask=Non
                                       workspace.numel() * workspace.element_size(),
                                       _stream_ptr(stream, x.device)), "sfn_dense4x_forward")
     return y, mask
+
+
+def sparse_ffn_backward(x, A, B, Wg, Wu, Wd, dy, bank: int = 64, k: int = 16,
+                        temperature: float = 1.0, want=("dx", "dA", "dB", "dWg", "dWu", "dWd"),
+                        workspace=None, stream=None) -> dict:
+    """Gradients of the layer for dy = dL/dy (bf16 inputs, float32 outputs),
+    with the soft surrogate gradient of the bank top-k (see
+    ``sfn_sparse_ffn_backward`` in include/sfn.h).  Returns a dict holding
+    the gradients named in ``want`` and the forward's ``mask``."""
+    torch = _torch()
+    for n, t in (("x", x), ("A", A), ("B", B), ("Wg", Wg), ("Wu", Wu), ("Wd", Wd), ("dy", dy)):
+        _dev(t, n)
+    T, d = x.shape
+    r = A.shape[0]
+    d_i = B.shape[0]
+    f32 = dict(dtype=torch.float32, device=x.device)
+    shapes = {"dx": (T, d), "dA": (r, d), "dB": (d_i, r), "dWg": (d_i, d), "dWu": (d_i, d),
+              "dWd": (d_i, d)}
+    out = {n: torch.empty(shapes[n], **f32) for n in want}
+    out["mask"] = torch.empty((T, max(d_i // max(bank, 1), 0)), dtype=torch.int64,
+                              device=x.device)
+    L = _capi.lib()
+    if workspace is None:
+        nbytes = int(L.sfn_backward_workspace_bytes(T, d, d_i, r, bank, k))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+
+    def ptr(n):
+        return out[n].data_ptr() if n in out else None
+
+    _capi.check(L.sfn_sparse_ffn_backward(
+        x.data_ptr(), A.data_ptr(), B.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), Wd.data_ptr(),
+        dy.data_ptr(), float(temperature), ptr("dx"), ptr("dA"), ptr("dB"), ptr("dWg"),
+        ptr("dWu"), ptr("dWd"), out["mask"].data_ptr(), T, d, d_i, r, bank, k,
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream, x.device)), "sfn_sparse_ffn_backward")
+    return out

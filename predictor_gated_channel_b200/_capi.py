@@ -45,6 +45,10 @@ SIGNATURES = {
     "sfn_dense4x_workspace_bytes": (_sz, [_i64, _ci, _ci, _ci, _ci]),
     "sfn_dense4x_forward": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _ci, _ci, _ci, _ci, _vp,
                                   _sz, _vp]),
+    "sfn_backward_workspace_bytes": (_sz, [_i64, _ci, _ci, _ci, _ci, _ci]),
+    "sfn_sparse_ffn_backward": (_ci, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp,
+                                      _vp, _vp, _vp, _vp, _vp, _i64, _ci, _ci, _ci, _ci, _ci,
+                                      _vp, _sz, _vp]),
     "sfn_timing_begin": (_ci, []),
     "sfn_device_errors": (_ci, [_vp, _ci]),
     "sfn_timing_end": (_ci, [_vp, _vp, _ci]),
@@ -61,7 +65,7 @@ class SfnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         msg = f"{where}: {status_string(status)}"
-        if status == SFN_ERR_CUDA:
+        if status in (SFN_ERR_CUDA, SFN_ERR_UNSUPPORTED):
             msg += f" ({lib().sfn_last_error_string().decode()})"
         super().__init__(msg)
 

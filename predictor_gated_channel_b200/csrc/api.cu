@@ -3,6 +3,7 @@
 // is enqueued, so an error status means nothing was written.
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <mutex>
@@ -572,6 +573,188 @@ sfn_status sfn_dense4x_forward(const void *x, const void *Wg, const void *Wu, co
   return cuda_status(e);
 }
 
+namespace {
+// Scratch of the backward.  tc: logits by the tensor-core kernels (the
+// forward's automatic choice for this T), h as bf16 hi | lo halves [T][2r];
+// otherwise h float32 plus a bf16 copy.
+struct BwdPlan {
+  bool tc;
+  int hsplit;
+  size_t off_h2, off_hpart, off_hf, off_hb, off_P, off_mask, off_tau, off_G, off_U, off_DA,
+      off_a, off_dg, off_du, off_dp, off_dH, off_dHb, total;
+};
+
+BwdPlan plan_bwd(const FwdShape &s) {
+  BwdPlan p{};
+  p.tc = use_tensor_path(s, SFN_PATH_AUTO);
+  p.hsplit = p.tc ? plan_tc(s).hsplit : 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t T = (size_t)s.T, r = (size_t)s.r, di = (size_t)s.d_i, nb = (size_t)s.n_banks;
+  p.off_h2 = take(p.tc ? T * 2 * r * 2 : 0);
+  p.off_hpart = take(p.tc && p.hsplit > 1 ? T * (size_t)p.hsplit * r * 4 : 0);
+  p.off_hf = take(p.tc ? 0 : T * r * 4);
+  p.off_hb = take(p.tc ? 0 : T * r * 2);
+  p.off_P = take(T * di * 4);
+  p.off_mask = take(T * nb * 8);
+  p.off_tau = take(T * nb * 4);
+  p.off_G = take(T * di * 4);
+  p.off_U = take(T * di * 4);
+  p.off_DA = take(T * di * 4);
+  p.off_a = take(T * di * 2);
+  p.off_dg = take(T * di * 2);
+  p.off_du = take(T * di * 2);
+  p.off_dp = take(T * di * 2);
+  p.off_dH = take(T * r * 4);
+  p.off_dHb = take(T * r * 2);
+  p.total = off;
+  return p;
+}
+
+sfn_status check_backward(int64_t T, int d, int d_i, int r, int bank, int k, float temp) {
+  sfn_status s0 = check_shape(T, d, d_i, r, bank, k);
+  if (s0 != SFN_OK) return s0;
+  if (!(temp > 0.f) || !std::isfinite(temp)) return SFN_ERR_INVALID_VALUE;
+  if ((s0 = check_limits(d, d_i, r)) != SFN_OK) return s0;
+  if ((s0 = check_rows(d, r, true)) != SFN_OK) return s0;
+  if (d_i % 4 != 0 || T > 0x7fffffffLL) return SFN_ERR_UNSUPPORTED;
+  return SFN_OK;
+}
+}  // namespace
+
+size_t sfn_backward_workspace_bytes(int64_t T, int d, int d_i, int r, int bank, int k) {
+  if (T == 0 || check_backward(T, d, d_i, r, bank, k, 1.f) != SFN_OK) return 0;
+  return plan_bwd(make_shape(T, d, d_i, r, bank, k, true)).total;
+}
+
+sfn_status sfn_sparse_ffn_backward(const void *x, const void *A, const void *B, const void *Wg,
+                                   const void *Wu, const void *Wd, const void *dy,
+                                   float temperature, float *dx, float *dA, float *dB,
+                                   float *dWg, float *dWu, float *dWd, uint64_t *mask,
+                                   int64_t T, int d, int d_i, int r, int bank, int k,
+                                   void *ws, size_t ws_bytes, sfn_stream_t stream) {
+  sfn_status s0 = check_backward(T, d, d_i, r, bank, k, temperature);
+  if (s0 != SFN_OK) return s0;
+  const char *why = nullptr;
+  if (!blas_available(&why)) {
+    t_last_error = why;
+    return SFN_ERR_UNSUPPORTED;
+  }
+  if (T == 0) return SFN_OK;
+  if (!x || !A || !B || !Wg || !Wu || !Wd || !dy) return SFN_ERR_INVALID_VALUE;
+  for (const void *q : {x, A, B, Wg, Wu, Wd, dy, (const void *)dx, (const void *)dA,
+                        (const void *)dB, (const void *)dWg, (const void *)dWu,
+                        (const void *)dWd})
+    if (q && !aligned(q, 16)) return SFN_ERR_MISALIGNED;
+  if (mask && !aligned(mask, 8)) return SFN_ERR_MISALIGNED;
+  FwdShape s = make_shape(T, d, d_i, r, bank, k, true);
+  const BwdPlan p = plan_bwd(s);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < p.total) return SFN_ERR_WORKSPACE;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return SFN_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  char *w = static_cast<char *>(ws);
+  auto F = [&](size_t off) { return reinterpret_cast<float *>(w + off); };
+  auto H = [&](size_t off) { return reinterpret_cast<uint16_t *>(w + off); };
+  float *P = F(p.off_P), *tau = F(p.off_tau), *G = F(p.off_G), *U = F(p.off_U);
+  float *DA = F(p.off_DA), *dH = F(p.off_dH);
+  uint16_t *a = H(p.off_a), *dg = H(p.off_dg), *du = H(p.off_du), *dp = H(p.off_dp);
+  uint16_t *dHb = H(p.off_dHb);
+  uint64_t *m = mask ? mask : reinterpret_cast<uint64_t *>(w + p.off_mask);
+  const int Ti = (int)T;
+
+  // 1. the forward's predictor (same kernels as the forward: same logits, same mask)
+  const uint16_t *hb;
+  int ldh;
+  cudaError_t e;
+  if (p.tc) {
+    uint16_t *h2 = H(p.off_h2);
+    if (p.hsplit > 1) {
+      float *hpart = F(p.off_hpart);
+      e = timed(SFN_STAGE_TC_H, st,
+                [&] { return launch_tc_h(s, dev, x, A, h2, hpart, p.hsplit, st); });
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_REDUCE, st, [&] {
+          return launch_reduce_partials(s, p.hsplit, hpart, h2, st, ReduceOut::kSplitH);
+        });
+    } else {
+      e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, nullptr, 1, st); });
+    }
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
+                [&] { return launch_tc_logits(s, dev, h2, B, P, nullptr, nullptr, st); });
+    hb = h2;  // the hi halves: bf16(h)
+    ldh = 2 * r;
+  } else {
+    float *hf = F(p.off_hf);
+    uint16_t *hbw = H(p.off_hb);
+    e = timed(SFN_STAGE_PRED_H, st, [&] {
+      return launch_pred_h(s, pred_tokens_per_cta(s), x, A, hf, false, st);
+    });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
+        return launch_logits_topk(s, pow2_tokens(T, 8), hf, B, P, nullptr, nullptr, nullptr,
+                                  dev.err, st);
+      });
+    if (e == cudaSuccess) e = launch_f32_to_bf16(hf, hbw, T * r, st);
+    hb = hbw;
+    ldh = r;
+  }
+  // 2. mask and thresholds
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_BWD_TAU, st,
+              [&] { return launch_bank_tau(P, m, tau, T, d_i, bank, k, st); });
+  BlasLock blas;
+  // 3. g, u (every channel) and da = Wd dy, float32 [T][d_i]
+  auto gemm = [&](bool ta, bool tb, int mm, int nn, int kk, const void *Am, int lda,
+                  const void *Bm, int ldb, float *C, int ldc, float beta) {
+    return blas_gemm_bf16(dev.device, st, ta, tb, mm, nn, kk, Am, lda, Bm, ldb, C, ldc, beta);
+  };
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_BWD_GEMM, st, [&] {
+      cudaError_t r1 = gemm(true, false, d_i, Ti, d, Wg, d, x, d, G, d_i, 0.f);
+      if (r1 == cudaSuccess) r1 = gemm(true, false, d_i, Ti, d, Wu, d, x, d, U, d_i, 0.f);
+      if (r1 == cudaSuccess) r1 = gemm(true, false, d_i, Ti, d, Wd, d, dy, d, DA, d_i, 0.f);
+      return r1;
+    });
+  // 4. the chain rule with the surrogate
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_BWD_ELEM, st, [&] {
+      return launch_bwd_elem(P, m, tau, G, U, DA, a, dg, du, dp, T, d_i, bank, temperature,
+                             st);
+    });
+  // 5. contractions back to the inputs
+  const bool need_dh = dA != nullptr || dx != nullptr;
+  if (e == cudaSuccess)
+    e = timed(SFN_STAGE_BWD_GEMM, st, [&] {
+      cudaError_t r1 = cudaSuccess;
+      if (dWd) r1 = gemm(false, true, d, d_i, Ti, dy, d, a, d_i, dWd, d, 0.f);
+      if (r1 == cudaSuccess && dWg) r1 = gemm(false, true, d, d_i, Ti, x, d, dg, d_i, dWg, d, 0.f);
+      if (r1 == cudaSuccess && dWu) r1 = gemm(false, true, d, d_i, Ti, x, d, du, d_i, dWu, d, 0.f);
+      if (r1 == cudaSuccess && dB) r1 = gemm(false, true, r, d_i, Ti, hb, ldh, dp, d_i, dB, r, 0.f);
+      if (r1 == cudaSuccess && need_dh)
+        r1 = gemm(false, false, r, Ti, d_i, B, r, dp, d_i, dH, r, 0.f);
+      return r1;
+    });
+  if (e == cudaSuccess && need_dh) e = launch_f32_to_bf16(dH, dHb, T * r, st);
+  if (e == cudaSuccess && need_dh)
+    e = timed(SFN_STAGE_BWD_GEMM, st, [&] {
+      cudaError_t r1 = cudaSuccess;
+      if (dA) r1 = gemm(false, true, d, r, Ti, x, d, dHb, r, dA, d, 0.f);
+      if (r1 == cudaSuccess && dx) {
+        r1 = gemm(false, false, d, Ti, d_i, Wg, d, dg, d_i, dx, d, 0.f);
+        if (r1 == cudaSuccess) r1 = gemm(false, false, d, Ti, d_i, Wu, d, du, d_i, dx, d, 1.f);
+        if (r1 == cudaSuccess) r1 = gemm(false, false, d, Ti, r, A, d, dHb, r, dx, d, 1.f);
+      }
+      return r1;
+    });
+  return cuda_status(e);
+}
+
 const char *sfn_stage_name(int stage) {
   switch (stage) {
     case SFN_STAGE_PRED_H: return "pred_h";
@@ -583,6 +766,9 @@ const char *sfn_stage_name(int stage) {
     case SFN_STAGE_TC_GATEUP: return "tc_gateup";
     case SFN_STAGE_TC_DOWN: return "tc_down";
     case SFN_STAGE_DENSE4X_GATEUP: return "dense4x_gateup";
+    case SFN_STAGE_BWD_TAU: return "bwd_tau";
+    case SFN_STAGE_BWD_ELEM: return "bwd_elem";
+    case SFN_STAGE_BWD_GEMM: return "bwd_gemm";
     case SFN_STAGE_BANK_TOPK: return "bank_topk";
   }
   return "unused";

@@ -1,6 +1,7 @@
 // sfn_internal.cuh -- device helpers and host launcher declarations shared by
 // the libsfn translation units.  Nothing here is part of the public ABI.
 #pragma once
+#include <mutex>
 
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -110,6 +111,48 @@ __device__ __forceinline__ uint64_t warp_bank_topk(uint32_t key0, uint32_t key1,
   return ((uint64_t)hi << 32) | lo;
 }
 
+// Descending compare-exchange on order keys.
+__device__ __forceinline__ void cex_desc(uint32_t &a, uint32_t &b) {
+  const uint32_t hi = max(a, b), lo = min(a, b);
+  a = hi;
+  b = lo;
+}
+
+// Bitonic network sorting s[OFF, OFF + N) in descending order.  Every index
+// is a compile-time constant (the stages are template-recursive), so the
+// array stays in registers.
+template <int OFF, int N, int SIZE, int STRIDE>
+struct BitonicStage {
+  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const int j = i ^ STRIDE;
+      if (j > i) {
+        if ((i & SIZE) == 0)
+          cex_desc(s[OFF + i], s[OFF + j]);
+        else
+          cex_desc(s[OFF + j], s[OFF + i]);
+      }
+    }
+    BitonicStage<OFF, N, SIZE, STRIDE / 2>::run(s);
+  }
+};
+template <int OFF, int N, int SIZE>
+struct BitonicStage<OFF, N, SIZE, 0> {
+  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
+};
+template <int OFF, int N, int SIZE>
+struct BitonicSort {
+  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
+    BitonicStage<OFF, N, SIZE, SIZE / 2>::run(s);
+    BitonicSort<OFF, N, SIZE * 2>::run(s);
+  }
+};
+template <int OFF, int N>
+struct BitonicSort<OFF, N, 2 * N> {
+  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
+};
+
 // --------------------------------------------------------------- host side
 struct DeviceInfo {
   int device = -1;
@@ -194,6 +237,29 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
 enum class ReduceOut { kY, kYLast, kSplitH };
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
                                    cudaStream_t st, ReduceOut kind = ReduceOut::kY);
+
+// ---------------------------------------------------------------- backward
+// cuBLAS, loaded at run time for the backward's plain GEMMs (bf16 operands,
+// float32 accumulate and output, column-major as cuBLAS sees it).  Hold a
+// BlasLock while enqueuing a sequence of blas_gemm_bf16 calls.
+bool blas_available(const char **why);
+class BlasLock {
+ public:
+  BlasLock();
+  ~BlasLock();
+ private:
+  std::lock_guard<std::mutex> lock_;
+};
+cudaError_t blas_gemm_bf16(int device, cudaStream_t st, bool ta, bool tb, int m, int n, int k,
+                           const void *A, int lda, const void *B, int ldb, float *C, int ldc,
+                           float beta);
+cudaError_t launch_bank_tau(const float *logits, uint64_t *mask, float *tau, int64_t T, int d_i,
+                            int bank, int k, cudaStream_t st);
+cudaError_t launch_bwd_elem(const float *P, const uint64_t *mask, const float *tau,
+                            const float *G, const float *U, const float *DA, uint16_t *a,
+                            uint16_t *dg, uint16_t *du, uint16_t *dp, int64_t T, int d_i,
+                            int bank, float temp, cudaStream_t st);
+cudaError_t launch_f32_to_bf16(const float *in, uint16_t *out, int64_t n, cudaStream_t st);
 
 // Scratch carve-up of the tensor-core path.
 struct TcPlan {

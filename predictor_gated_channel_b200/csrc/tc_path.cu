@@ -103,48 +103,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return (uint32_t)f32_to_bf16_bits(a) | ((uint32_t)f32_to_bf16_bits(b) << 16);
 }
 
-// Descending compare-exchange on order keys.
-__device__ __forceinline__ void cex_desc(uint32_t &a, uint32_t &b) {
-  const uint32_t hi = max(a, b), lo = min(a, b);
-  a = hi;
-  b = lo;
-}
-
-// Bitonic network sorting s[OFF, OFF + N) in descending order.  Every index
-// is a compile-time constant (the stages are template-recursive), so the
-// array stays in registers.
-template <int OFF, int N, int SIZE, int STRIDE>
-struct BitonicStage {
-  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-      const int j = i ^ STRIDE;
-      if (j > i) {
-        if ((i & SIZE) == 0)
-          cex_desc(s[OFF + i], s[OFF + j]);
-        else
-          cex_desc(s[OFF + j], s[OFF + i]);
-      }
-    }
-    BitonicStage<OFF, N, SIZE, STRIDE / 2>::run(s);
-  }
-};
-template <int OFF, int N, int SIZE>
-struct BitonicStage<OFF, N, SIZE, 0> {
-  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
-};
-template <int OFF, int N, int SIZE>
-struct BitonicSort {
-  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
-    BitonicStage<OFF, N, SIZE, SIZE / 2>::run(s);
-    BitonicSort<OFF, N, SIZE * 2>::run(s);
-  }
-};
-template <int OFF, int N>
-struct BitonicSort<OFF, N, 2 * N> {
-  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
-};
-
 // s[A..A+16) and s[B..B+16) sorted descending -> s[A..A+16) = the 16 largest
 // of both, sorted descending (max with the reversed other list gives a
 // bitonic sequence, which a half-cleaner cascade sorts).

@@ -160,3 +160,29 @@ def test_path_selector_validation(L):
     assert L.sfn_sparse_ffn_forward_path(*bad, _capi.SFN_PATH_TENSOR, FAKE, need, None) == \
         _capi.SFN_ERR_UNSUPPORTED
     assert L.sfn_last_error_string() is not None
+
+
+def test_backward_validation(L):
+    need = L.sfn_backward_workspace_bytes(4, 4096, 14336, 448, 64, 16)
+    assert need > 0 and need % 256 == 0
+    assert L.sfn_backward_workspace_bytes(0, 4096, 14336, 448, 64, 16) == 0
+    assert L.sfn_backward_workspace_bytes(4, 4096, 14336, 448, 64, 0) == 0
+    ins = [FAKE] * 7
+    grads = [FAKE] * 6 + [None]
+
+    def bwd(temp=1.0, T=4, d=4096, d_i=14336, r=448, bank=64, k=16, ins=ins, grads=grads,
+            ws=FAKE, ws_bytes=need):
+        return L.sfn_sparse_ffn_backward(*ins, temp, *grads, T, d, d_i, r, bank, k, ws,
+                                         ws_bytes, None)
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert bwd(temp=bad) == _capi.SFN_ERR_INVALID_VALUE
+    assert bwd(k=0) == _capi.SFN_ERR_INVALID_VALUE
+    assert bwd(d_i=14330, bank=10, k=2) == _capi.SFN_ERR_UNSUPPORTED  # d_i % 4 != 0
+    assert bwd(T=0, ws=None, ws_bytes=0) == _capi.SFN_OK
+    assert bwd(ws_bytes=need - 256) == _capi.SFN_ERR_WORKSPACE
+    p = list(ins)
+    p[6] = None  # dy
+    assert bwd(ins=p) == _capi.SFN_ERR_INVALID_VALUE
+    g = list(grads)
+    g[3] = FAKE + 4  # dWg misaligned
+    assert bwd(grads=g) == _capi.SFN_ERR_MISALIGNED
