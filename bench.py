@@ -56,6 +56,10 @@ def parse_args(argv=None):
                     help="sfn: the predictor-gated sparse FFN; dense4x: the pages' post-hoc "
                          "comparison (dense gate/up, amplitude top-k, sparse down); backward: "
                          "the layer's backward with the surrogate top-k gradient")
+    ap.add_argument("--shard", default="tokens", choices=["tokens", "banks"],
+                    help="tokens: every rank runs the whole layer on its own tokens (weak "
+                         "scaling); banks: the ranks split one layer's banks and sum their "
+                         "float32 partial outputs with an all-reduce (strong scaling)")
     ap.add_argument("--temperature", type=float, default=1.0,
                     help="surrogate temperature of --method backward")
     ap.add_argument("--path", default="auto", choices=["auto", "cuda_core", "tensor"],
@@ -280,9 +284,23 @@ def run_sfn(args, rank, world, local):
     S = rotation_layers(args.workload)
     peaks = load_peaks()
 
-    layers = [make_layer_device(wl, dev, seed=rank, layer=i) for i in range(S)]
-    xs = [make_tokens_device(wl, dev, seed=rank, layer=i) for i in range(S)]
-    ys = [torch.empty((T, wl.d), dtype=wl.torch_dtype, device=dev) for _ in range(S)]
+    shard = args.shard == "banks"
+    if shard and (args.method != "sfn" or wl.dtype != "bf16"):
+        raise SystemExit("bench.py: --shard banks runs the bf16 forward")
+    # bank shards: every rank holds the same layer and tokens and keeps its banks
+    seed = 0 if shard else rank
+    layers = [make_layer_device(wl, dev, seed=seed, layer=i) for i in range(S)]
+    xs = [make_tokens_device(wl, dev, seed=seed, layer=i) for i in range(S)]
+    wl_full = wl
+    if shard:
+        b0, b1 = sfn.bank_shard(wl.n_banks, rank, world)
+        rows = slice(b0 * wl.bank, b1 * wl.bank)
+        for lay in layers:
+            for n in ("B", "Wg", "Wu", "Wd"):
+                lay[n] = lay[n][rows]
+        wl = wl.with_(d_i=(b1 - b0) * wl.bank)
+    ys = [torch.empty((T, wl.d), dtype=torch.float32 if shard else wl.torch_dtype, device=dev)
+          for _ in range(S)]
     ms = [torch.empty((T, wl.n_banks), dtype=torch.int64, device=dev) for _ in range(S)]
     dense4x = args.method == "dense4x"
     backward = args.method == "backward"
@@ -319,6 +337,13 @@ def run_sfn(args, rank, world, local):
             rc = L.sfn_dense4x_forward(ptrs[0], ptrs[3], ptrs[4], ptrs[5], ptrs[6], ptrs[7], T,
                                        wl.d, wl.d_i, wl.bank, wl.k, ws.data_ptr(), ws_bytes,
                                        st_ptr)
+        elif shard:
+            rc = L.sfn_sparse_ffn_forward_partial(*ptrs, path_id, ws.data_ptr(), ws_bytes,
+                                                  st_ptr)
+            if world > 1:
+                _capi.check(rc, "sfn_sparse_ffn_forward_partial")
+                import torch.distributed as dist
+                dist.all_reduce(ys[i])  # sum of the ranks' partial outputs
         elif wl.dtype == "bf16":
             rc = L.sfn_sparse_ffn_forward_path(*ptrs, path_id, ws.data_ptr(), ws_bytes, st_ptr)
         else:
@@ -342,11 +367,24 @@ def run_sfn(args, rank, world, local):
                 call(i % S, stream.cuda_stream)
         return g, L.sfn_kernel_launch_count() - c0
 
-    g_full, launches_full = capture(S)
-    g_rem, launches_rem = capture(K % S)
-    launches_per_step = launches_full / S
+    eager = shard and world > 1  # steps with a collective run eagerly
+    if eager:
+        g_full = g_rem = None
+        c0 = L.sfn_kernel_launch_count()
+        with torch.cuda.stream(stream):
+            call(0, stream.cuda_stream)
+        stream.synchronize()
+        launches_per_step = L.sfn_kernel_launch_count() - c0
+    else:
+        g_full, launches_full = capture(S)
+        g_rem, launches_rem = capture(K % S)
+        launches_per_step = launches_full / S
 
     def replay(nsteps):
+        if eager:
+            for j in range(nsteps):
+                call(j % S, stream.cuda_stream)
+            return
         for _ in range(nsteps // S):
             g_full.replay()
         if nsteps % S:
@@ -360,13 +398,17 @@ def run_sfn(args, rank, world, local):
 
     # warm-up: W untimed steps, then keep the GPU loaded ~1 s so clocks settle
     with torch.cuda.stream(stream):
-        for _ in range(W // S):
-            g_full.replay()
-        for i in range(W % S):
-            call(i, stream.cuda_stream)
-        t_settle = time.time()
-        while time.time() - t_settle < args.settle:
-            g_full.replay()
+        if eager:
+            # a fixed number of steps: every rank must make the same collective calls
+            replay(W + int(args.settle * 1000))
+        else:
+            for _ in range(W // S):
+                g_full.replay()
+            for i in range(W % S):
+                call(i, stream.cuda_stream)
+            t_settle = time.time()
+            while time.time() - t_settle < args.settle:
+                g_full.replay()
         stream.synchronize()
 
     if world > 1:
@@ -441,7 +483,7 @@ def run_sfn(args, rank, world, local):
 
     # end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e and not backward:
+    if not args.no_e2e and not backward and not shard:
         n_e2e = min(K, 300 if T <= 64 else 10)
         x_host = [xs[i].cpu().pin_memory() for i in range(S)]
         y_host = torch.empty((T, wl.d), dtype=wl.torch_dtype).pin_memory()
@@ -492,7 +534,9 @@ def run_sfn(args, rank, world, local):
     if rank != 0:
         return None
 
-    value = world * T * K / (elapsed_ms_max * 1e-3)
+    # token replicas: every rank processes its own T tokens; bank shards: the
+    # ranks share one batch of T tokens
+    value = (1 if shard else world) * T * K / (elapsed_ms_max * 1e-3)
     # the path's algorithmic minimum: predictor weights, kept rows, x and y
     if dense4x:
         step_bytes = sum(work[n]["bytes"] for n in ("dense4x_gateup", "tc_down"))
@@ -505,18 +549,23 @@ def run_sfn(args, rank, world, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": elapsed_ms_max / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic",
         "config": {
-            "workload": f"{wl.name}: T={T} d={wl.d} d_i={wl.d_i} r={wl.r} bank={wl.bank} "
-                        f"k={wl.k} {wl.dtype}",
-            "T": T, "d": wl.d, "d_i": wl.d_i, "r": wl.r, "bank": wl.bank, "k": wl.k,
-            "method": args.method,
+            "workload": f"{wl_full.name}: T={T} d={wl_full.d} d_i={wl_full.d_i} r={wl_full.r} "
+                        f"bank={wl_full.bank} k={wl_full.k} {wl_full.dtype}",
+            "T": T, "d": wl_full.d, "d_i": wl_full.d_i, "r": wl_full.r, "bank": wl_full.bank,
+            "k": wl_full.k, "method": args.method,
             "l2": (f"inputs larger than L2: steps rotate over {S} distinct layers "
                    f"({S * sum(v.numel() * v.element_size() for v in layers[0].values()) / 1e9:.2f}"
                    " GB of weights)"),
-            "parallelism": f"replica x{world} (token batches independent)",
+            "parallelism": (f"bank shards x{world} (all-reduce of float32 partial y)" if shard
+                            else f"replica x{world} (token batches independent)"),
             "path": args.path,
-            "timing": "CUDA graph replay of the steps, CUDA events on the launching stream",
+            "timing": ("eager steps (each ends in an all-reduce)" if eager else
+                       "CUDA graph replay of the steps") + ", CUDA events on the launching stream",
+            **({"shard": f"rank 0 holds banks {b0}..{b1 - 1}; roofline figures are per rank"}
+               if shard else {}),
         },
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": unit, "frac": achieved / peak, "traffic": traffic,

@@ -223,6 +223,28 @@ sfn_status sfn_sparse_ffn_forward_path(const void *x, const void *A, const void 
                                        size_t workspace_bytes, sfn_stream_t stream);
 
 /*
+ * One bank shard of the layer, for splitting a layer's banks over devices
+ * (banks are independent through the top-k and the three projections, so a
+ * device that holds banks [b0, b1) computes their contribution to y and the
+ * devices sum their partial outputs, e.g. with an all-reduce).
+ *
+ * B, Wg, Wu and Wd point at the shard's first row (channel b0 * bank) and
+ * d_i is the shard's channel count (a multiple of bank); A and x are the
+ * whole predictor factor and input.  y_partial [T][d] receives, in float32
+ * and without rounding, sum over the shard's kept channels of a_j Wd[j];
+ * mask (may be NULL) the shard's mask words.  The sum of y_partial over a
+ * partition of the banks, rounded to bf16, is the layer's y.  bf16 inputs;
+ * scratch sfn_workspace_bytes(T, d, d_i (the shard's), r, bank, k,
+ * SFN_DTYPE_BF16); path and errors as sfn_sparse_ffn_forward_path.
+ */
+sfn_status sfn_sparse_ffn_forward_partial(const void *x, const void *A, const void *B,
+                                          const void *Wg, const void *Wu, const void *Wd,
+                                          float *y_partial, uint64_t *mask, int64_t T, int d,
+                                          int d_i, int r, int bank, int k, sfn_path path,
+                                          void *workspace, size_t workspace_bytes,
+                                          sfn_stream_t stream);
+
+/*
  * The pages' "Dense-4x" comparison (gist.science summary, "Resultaten": a
  * dense model made 4x sparse post hoc from the activation amplitude).
  * Reading: the standard SwiGLU FFN without a predictor -- act_j =

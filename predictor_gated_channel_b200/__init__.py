@@ -162,6 +162,43 @@ def sparse_ffn_forward(x, A, B, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None,
     return y, mask
 
 
+def bank_shard(n_banks: int, rank: int, world: int) -> tuple:
+    """Banks [b0, b1) of shard ``rank`` of ``world``: contiguous, sizes differing by
+    at most one, covering every bank once."""
+    if not 0 <= rank < world:
+        raise ValueError("bank_shard: rank outside [0, world)")
+    return n_banks * rank // world, n_banks * (rank + 1) // world
+
+
+def sparse_ffn_forward_partial(x, A, B, Wg, Wu, Wd, bank: int = 64, k: int = 16,
+                               y_partial=None, mask=None, workspace=None, path: str = "auto",
+                               stream=None):
+    """One bank shard of the layer (bf16): B, Wg, Wu, Wd hold only the shard's
+    rows.  Returns (y_partial float32 [T, d], mask int64 [T, shard banks]); the
+    sum of y_partial over a partition of the banks is the layer's y before
+    rounding."""
+    torch = _torch()
+    for n, t in (("x", x), ("A", A), ("B", B), ("Wg", Wg), ("Wu", Wu), ("Wd", Wd)):
+        _dev(t, n)
+    T, d = x.shape
+    r, d_i = A.shape[0], B.shape[0]
+    if y_partial is None:
+        y_partial = torch.empty((T, d), dtype=torch.float32, device=x.device)
+    if mask is None:
+        mask = torch.empty((T, max(d_i // max(bank, 1), 0)), dtype=torch.int64,
+                           device=x.device)
+    if workspace is None:
+        nbytes = workspace_bytes(T, d, d_i, r, bank, k, x.dtype)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    L = _capi.lib()
+    _capi.check(L.sfn_sparse_ffn_forward_partial(
+        x.data_ptr(), A.data_ptr(), B.data_ptr(), Wg.data_ptr(), Wu.data_ptr(), Wd.data_ptr(),
+        y_partial.data_ptr(), mask.data_ptr(), T, d, d_i, r, bank, k, PATHS[path],
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream, x.device)), "sfn_sparse_ffn_forward_partial")
+    return y_partial, mask
+
+
 def dense4x_forward(x, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None, mask=None,
                     workspace=None, stream=None):
     """The Dense-4x comparison (post-hoc amplitude top-k of the SwiGLU

@@ -40,6 +40,7 @@ SIGNATURES = {
     "sfn_sparse_ffn_forward_ws": (_ci, _FWD + [_vp, _sz, _vp]),
     "sfn_sparse_ffn_forward_static": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_path": (_ci, _FWD + [_ci, _vp, _sz, _vp]),
+    "sfn_sparse_ffn_forward_partial": (_ci, _FWD + [_ci, _vp, _sz, _vp]),
     "sfn_sparse_ffn_forward_f32": (_ci, _FWD + [_vp]),
     "sfn_sparse_ffn_forward_f32_ws": (_ci, _FWD + [_vp, _sz, _vp]),
     "sfn_dense4x_workspace_bytes": (_sz, [_i64, _ci, _ci, _ci, _ci]),

@@ -267,7 +267,8 @@ size_t workspace_for(const FwdShape &s) {
 sfn_status forward_impl(const void *x, const void *A, const void *B, const void *Wg,
                         const void *Wu, const void *Wd, void *y, uint64_t *mask, int64_t T,
                         int d, int d_i, int r, int bank, int k, bool bf16, sfn_path path,
-                        void *ws, size_t ws_bytes, bool own_ws, cudaStream_t st) {
+                        void *ws, size_t ws_bytes, bool own_ws, cudaStream_t st,
+                        bool y_f32 = false) {
   sfn_status s0 = check_shape(T, d, d_i, r, bank, k);
   if (s0 != SFN_OK) return s0;
   if (path != SFN_PATH_AUTO && path != SFN_PATH_CUDA_CORE && path != SFN_PATH_TENSOR)
@@ -325,11 +326,13 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
         e = timed(SFN_STAGE_TC_DOWN, st,
                   [&] { return launch_tc_down(s, dev, act, Wd, part, p.ksplit, st); });
       if (e == cudaSuccess)
-        e = timed(SFN_STAGE_REDUCE, st,
-                  [&] { return launch_reduce_partials(s, p.ksplit, part, y, st); });
+        e = timed(SFN_STAGE_REDUCE, st, [&] {
+          return launch_reduce_partials(s, p.ksplit, part, y, st,
+                                        y_f32 ? ReduceOut::kYF32 : ReduceOut::kY);
+        });
     } else if (e == cudaSuccess) {
       e = timed(SFN_STAGE_TC_DOWN, st,
-                [&] { return launch_tc_down(s, dev, act, Wd, y, 1, st); });
+                [&] { return launch_tc_down(s, dev, act, Wd, y, 1, st, y_f32); });
     }
   } else {
     const GatherPlan p = plan_gather(s);
@@ -350,7 +353,10 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
       });
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_REDUCE, st,
-                [&] { return launch_reduce_partials(s, p.cpt, partial, y, st, ReduceOut::kYLast); });
+                [&] {
+                  return launch_reduce_partials(s, p.cpt, partial, y, st,
+                                                y_f32 ? ReduceOut::kYF32 : ReduceOut::kYLast);
+                });
   }
   if (own_ws) {
     cudaError_t ef = cudaFreeAsync(ws, st);
@@ -459,6 +465,16 @@ sfn_status sfn_sparse_ffn_forward_path(const void *x, const void *A, const void 
                                        size_t workspace_bytes, sfn_stream_t stream) {
   return forward_impl(x, A, B, Wg, Wu, Wd, y, mask, T, d, d_i, r, bank, k, true, path,
                       workspace, workspace_bytes, false, (cudaStream_t)stream);
+}
+
+sfn_status sfn_sparse_ffn_forward_partial(const void *x, const void *A, const void *B,
+                                          const void *Wg, const void *Wu, const void *Wd,
+                                          float *y_partial, uint64_t *mask, int64_t T, int d,
+                                          int d_i, int r, int bank, int k, sfn_path path,
+                                          void *workspace, size_t workspace_bytes,
+                                          sfn_stream_t stream) {
+  return forward_impl(x, A, B, Wg, Wu, Wd, y_partial, mask, T, d, d_i, r, bank, k, true, path,
+                      workspace, workspace_bytes, false, (cudaStream_t)stream, true);
 }
 
 sfn_status sfn_sparse_ffn_forward_f32(const float *x, const float *A, const float *B,
@@ -684,9 +700,10 @@ sfn_status sfn_sparse_ffn_backward(const void *x, const void *A, const void *B, 
     } else {
       e = timed(SFN_STAGE_TC_H, st, [&] { return launch_tc_h(s, dev, x, A, h2, nullptr, 1, st); });
     }
+    // logits, mask and thresholds from one GEMM epilogue
     if (e == cudaSuccess)
       e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
-                [&] { return launch_tc_logits(s, dev, h2, B, P, nullptr, nullptr, st); });
+                [&] { return launch_tc_logits_tau(s, dev, h2, B, P, m, tau, st); });
     hb = h2;  // the hi halves: bf16(h)
     ldh = 2 * r;
   } else {
@@ -704,8 +721,8 @@ sfn_status sfn_sparse_ffn_backward(const void *x, const void *A, const void *B, 
     hb = hbw;
     ldh = r;
   }
-  // 2. mask and thresholds
-  if (e == cudaSuccess)
+  // 2. mask and thresholds (the tensor-core logits epilogue already wrote them)
+  if (e == cudaSuccess && !p.tc)
     e = timed(SFN_STAGE_BWD_TAU, st,
               [&] { return launch_bank_tau(P, m, tau, T, d_i, bank, k, st); });
   BlasLock blas;

@@ -40,12 +40,6 @@ namespace {
 constexpr int kElemThreads = 256;
 constexpr int kTauThreads = 128;
 
-// Float value of an order key (the inverse of order_key for numbers; -0
-// comes back as +0).
-__device__ __forceinline__ float key_value(uint32_t key) {
-  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
-}
-
 // One thread per (token, bank): the bank's logits become order keys (padding
 // past `bank` gets key 0, below every number), a register bitonic network
 // sorts a copy, the k-th and (k+1)-th keys give the threshold, and the mask

@@ -348,6 +348,8 @@ cudaError_t reduce_c(const FwdShape &s, int n, int cpt, const float *partial, vo
   const dim3 grid((unsigned)blocks), block(kReduceThreads);
   if (kind == ReduceOut::kSplitH)
     return launch_pdl(k_reduce_partials<C, 2, false>, grid, block, 0, st, partial, out, n, cpt);
+  if (kind == ReduceOut::kYF32)
+    return launch_pdl(k_reduce_partials<C, 0, false>, grid, block, 0, st, partial, out, n, cpt);
   if (kind == ReduceOut::kYLast) {
     if (s.bf16)
       return launch_pdl(k_reduce_partials<C, 1, true>, grid, block, 0, st, partial, out, n, cpt);

@@ -80,6 +80,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Float value of an order key (the inverse of order_key for numbers; -0
+// comes back as +0).
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 // Hard top-k of one bank (bank <= 64) held by a warp: lane l holds the keys
 // of channels l (key0) and l + 32 (key1).  Channel i ranks below channel j
 // when key_j > key_i, or key_j == key_i and j < i; a channel is kept when
@@ -234,7 +240,9 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
 // hi/lo halves of h ([T][2r], "split").  kYLast: y, from the last kernel of
 // a call on the CUDA-core path, which lets the stream's next kernel start
 // its (weights-only) prologue at once.
-enum class ReduceOut { kY, kYLast, kSplitH };
+// kYF32: y as float32 whatever the input type (partial outputs of a bank
+// shard, summed across devices before rounding).
+enum class ReduceOut { kY, kYLast, kYF32, kSplitH };
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
                                    cudaStream_t st, ReduceOut kind = ReduceOut::kY);
 
@@ -282,7 +290,11 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
 cudaError_t launch_tc_dense4x_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
                                      const void *Wg, const void *Wu, uint64_t *mask,
                                      uint16_t *act, cudaStream_t st);
+cudaError_t launch_tc_logits_tau(const FwdShape &s, const DeviceInfo &dev, const uint16_t *h2,
+                                 const void *B, float *logits, uint64_t *mask, float *tau,
+                                 cudaStream_t st);
 cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
-                           const void *Wd, void *y, int ksplit, cudaStream_t st);
+                           const void *Wd, void *y, int ksplit, cudaStream_t st,
+                           bool f32_out = false);
 
 }  // namespace sfn

@@ -42,7 +42,7 @@ namespace {
 constexpr int kBM = 128;                       // token rows per tile (UMMA M)
 constexpr int kBK = 64;                        // K per stage: 128-byte rows
 constexpr uint32_t kTileA = kBM * kBK * 2;     // 16 KB
-constexpr int kThreadsTc = 192;
+
 constexpr int kAccCols = 256;                  // TMEM columns per accumulator
 constexpr size_t kMaxDynSmem = 232448;            // 227 KB per CTA on sm_100
 constexpr int kGroupM = 8;                     // tile rasterisation group
@@ -69,6 +69,9 @@ struct TcParams {
   float *sig;             // top-k: written; gate/up: read  ([T][n_banks][k])
   int ld_out;             // elements per output row
   int r, k, n_banks;
+  bool f32_out;           // down: float32 y (no bf16 rounding), ksplit == 1
+  float *tau;             // top-k, if set: threshold per (token, bank) and float32 logits
+                          // into out ([T][ld_out]); sig may then be null
   unsigned *err;
 };
 
@@ -77,6 +80,10 @@ struct EpiTraits {
   static constexpr int kNumA = (kEpi == kEpiLogits || kEpi == kEpiTopk) ? 2 : 1;
   static constexpr bool kBMnMajor = (kEpi == kEpiDown);
   static constexpr bool kGateUpB = (kEpi == kEpiGateUp || kEpi == kEpiDense4x);
+  // epilogue warps: two per TMEM lane quadrant for the top-k (its sorting
+  // networks, not the MMAs, bound that GEMM), splitting the tile's banks
+  static constexpr int kEpiWarps = (kEpi == kEpiTopk) ? 8 : 4;
+  static constexpr int kThreads = (2 + kEpiWarps) * 32;
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &mb,
@@ -124,7 +131,6 @@ __device__ __forceinline__ float sigmoid_fast(float z) {
   return __fdividef(1.0f, 1.0f + __expf(-z));
 }
 
-constexpr int kStageRow = 65;  // floats per epilogue thread row (k <= 64, padded)
 
 // k-th largest of 64 order keys (s is reordered), and the number of keys
 // strictly above it.
@@ -192,7 +198,7 @@ __device__ __forceinline__ void bank_threshold(uint32_t taddr, int k, uint32_t &
 }
 
 template <int kEpi>
-__global__ void __launch_bounds__(kThreadsTc, 1)
+__global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
               const __grid_constant__ CUtensorMap tB2, const TcParams p) {
   using Tr = EpiTraits<kEpi>;
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4 * 32);
+      mbar_init(&tempty[i], Tr::kEpiWarps * 32);
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -318,6 +324,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;           // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;    // token row inside the tile
+    const int half_id = (warp - 2) >> 2;  // which of a quadrant's epilogue warps
     uint32_t lt = 0;
     for (int unit = blockIdx.x; unit < total; unit += gridDim.x, ++lt) {
       int mb, nb, kb0, kb1;
@@ -363,7 +370,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           tmem_ld_wait();
           if (valid) {
             const int col = nb * p.bn + c0;
-            if (kEpi != kEpiDown || p.ksplit > 1) {
+            if (kEpi != kEpiDown || p.ksplit > 1 || p.f32_out) {
               // fp32 logits, or fp32 partial sums [T][ksplit][ld_out]
               const int64_t orow = (p.ksplit > 1) ? t * p.ksplit + unit % p.ksplit : t;
               uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<float *>(p.out) +
@@ -389,20 +396,29 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         // bn/64 banks of 64 channels per tile.  The mask pass is branch-free: the
         // logits of kept channels are compacted, in channel order, into this
         // thread's staging row; sigma is then evaluated for those k only.
-        float *stg = stage_rows_smem + row * kStageRow;
+        const int srow = p.k | 1;  // staged floats per thread row (odd: no bank conflicts)
+        float *stg = stage_rows_smem + (half_id * kBM + row) * srow;
         const int banks_per_tile = p.bn / 64;
-        for (int bl = 0; bl < banks_per_tile; ++bl) {
+        for (int bl = half_id; bl < banks_per_tile; bl += Tr::kEpiWarps / 4) {
           uint32_t tau;
           int gt;
           bank_threshold(taddr + bl * 64, p.k, tau, gt);
           const int need = p.k - gt;
+          const int bank = nb * banks_per_tile + bl;
           int eq = 0, cnt = 0;
-          uint32_t bits[2];
+          uint32_t bits[2], rest = 0u;  // rest: largest key not kept
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(taddr + bl * 64 + half * 32, v);
             tmem_ld_wait();
+            if (p.tau != nullptr && valid) {
+              uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<float *>(p.out) +
+                                                     t * p.ld_out + bank * 64 + half * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
             uint32_t b = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -410,14 +426,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
               const bool take = (key > tau) | ((key == tau) & (eq < need));
               eq += (key == tau);
               b |= (uint32_t)take << i;
+              rest = max(rest, take ? 0u : key);
               if (take) stg[cnt] = __uint_as_float(v[i]);
               cnt += take;
             }
             bits[half] = b;
           }
-          const int bank = nb * banks_per_tile + bl;
-          if (valid) {
-            p.mask[t * p.n_banks + bank] = ((uint64_t)bits[1] << 32) | bits[0];
+          if (valid && p.tau != nullptr)
+            p.tau[t * p.n_banks + bank] = (p.k < 64)
+                                              ? 0.5f * (key_value(tau) + key_value(rest))
+                                              : __int_as_float(0x7fc00000);
+          if (valid) p.mask[t * p.n_banks + bank] = ((uint64_t)bits[1] << 32) | bits[0];
+          if (valid && p.sig != nullptr) {
             float *sig_out = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
             if ((p.k & 3) == 0) {
               for (int s4 = 0; s4 < p.k; s4 += 4)
@@ -576,7 +596,8 @@ cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtens
   using Tr = EpiTraits<kEpi>;
   const uint32_t b_bytes = (kEpi == kEpiDown) ? 32768u : (uint32_t)p.bn * 128u;
   p.stage_bytes = Tr::kNumA * kTileA + b_bytes;
-  const size_t epi_bytes = (kEpi == kEpiTopk) ? (size_t)kBM * kStageRow * sizeof(float) : 0;
+  const size_t epi_bytes =
+      (kEpi == kEpiTopk) ? (size_t)(Tr::kEpiWarps / 4) * kBM * (p.k | 1) * sizeof(float) : 0;
   // as many stages as fit beside the alignment slack, barriers and staging
   const size_t fixed = 1024 + 256 + epi_bytes;
   p.stages = (int)(((size_t)kMaxDynSmem - fixed) / p.stage_bytes);
@@ -590,7 +611,7 @@ cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtens
   if (e != cudaSuccess) return e;
   const int total = p.tiles_m * p.tiles_n * p.ksplit;
   const int grid = total < num_sms ? total : num_sms;
-  e = launch_pdl(kern, dim3(grid), dim3(kThreadsTc), smem, st, tA, tB, tB2, p);
+  e = launch_pdl(kern, dim3(grid), dim3(Tr::kThreads), smem, st, tA, tB, tB2, p);
   count_launches(1);
   return e;
 }
@@ -718,6 +739,29 @@ cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uin
   return launch_tc<kEpiTopk>(mH, mB, mB, p, dev.num_sms, st);
 }
 
+// G2 for the backward: logits (float32 [T][d_i]), mask and each bank's
+// threshold (midpoint of its k-th and (k+1)-th logits) from the same epilogue.
+cudaError_t launch_tc_logits_tau(const FwdShape &s, const DeviceInfo &dev, const uint16_t *h2,
+                                 const void *B, float *logits, uint64_t *mask, float *tau,
+                                 cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  const int tiles_m = (int)((s.T + kBM - 1) / kBM);
+  const int bn = pick_bn(tiles_m, s.d_i, {256, 128, 64}, dev.num_sms);
+  CUtensorMap mH, mB;
+  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, kBM) || !make_map(&mB, B, s.r, s.d_i, 64, bn))
+    return cudaErrorInvalidValue;
+  TcParams p = base_params(s, dev);
+  p.tiles_n = s.d_i / bn;
+  p.k_blocks = s.r / kBK;
+  p.bn = bn;
+  p.out = logits;
+  p.ld_out = s.d_i;
+  p.mask = mask;
+  p.sig = nullptr;
+  p.tau = tau;
+  return launch_tc<kEpiTopk>(mH, mB, mB, p, dev.num_sms, st);
+}
+
 // G3: [G | U] = X [Wg; Wu]^T -> act = sigma(p) g u on kept channels, 0 elsewhere.
 cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
                              const void *Wg, const void *Wu, const uint64_t *mask,
@@ -771,7 +815,7 @@ cudaError_t launch_tc_dense4x_gateup(const FwdShape &s, const DeviceInfo &dev, c
 // G4: Y = act Wd, with Wd [d_i][d] read as an MN-major B operand.  With
 // ksplit > 1, y receives fp32 partial sums [T][ksplit][d] instead.
 cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
-                           const void *Wd, void *y, int ksplit, cudaStream_t st) {
+                           const void *Wd, void *y, int ksplit, cudaStream_t st, bool f32_out) {
   if (!encoder()) return cudaErrorNotSupported;
   CUtensorMap mAct, mD;
   if (!make_map(&mAct, act, s.d_i, s.T, 64, kBM) || !make_map(&mD, Wd, s.d, s.d_i, 64, 64))
@@ -783,6 +827,7 @@ cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint1
   p.bn = 256;
   p.out = y;
   p.ld_out = s.d;
+  p.f32_out = f32_out;
   return launch_tc<kEpiDown>(mAct, mD, mD, p, dev.num_sms, st);
 }
 

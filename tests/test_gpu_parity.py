@@ -300,3 +300,31 @@ def test_dense4x_against_oracle(T, full_layer):
     y_ref, _ = oracle.dense4x(xs, host["Wg"], host["Wu"], host["Wd"], 64, 16, mask=gm)
     err = parity.y_error(y.float().cpu().numpy()[rows], y_ref)
     assert err <= parity.Y_TOL["bf16"], err
+
+
+@pytest.mark.parametrize("T,world", [(1, 2), (64, 2), (3, 3)])
+def test_bank_shards_sum_to_the_layer(T, world, full_layer):
+    """Bank-sharded layer on one device: every shard's float32 partial y from
+    its own rows, summed, equals the layer (oracle on the concatenated GPU
+    masks); the shard masks concatenate to a valid mask of the whole layer."""
+    wl, host, dev = full_layer
+    x = make_tokens(wl, T=T, seed=11)
+    xd = x.to(DEV)
+    total = torch.zeros((T, wl.d), dtype=torch.float32, device=DEV)
+    masks = []
+    for rank in range(world):
+        b0, b1 = sfn.bank_shard(wl.n_banks, rank, world)
+        rows = slice(b0 * wl.bank, b1 * wl.bank)
+        yp, m = sfn.sparse_ffn_forward_partial(xd, dev["A"], dev["B"][rows], dev["Wg"][rows],
+                                               dev["Wu"][rows], dev["Wd"][rows], bank=wl.bank,
+                                               k=wl.k)
+        total += yp
+        masks.append(m)
+    torch.cuda.synchronize()
+    gm = parity.to_u64(torch.cat(masks, dim=1))
+    logits = oracle.predict(x, host["A"], host["B"])
+    parity.check_mask(gm, logits, wl.bank, wl.k)
+    ref = oracle.forward_given_mask(x, logits, gm, host["Wg"], host["Wu"], host["Wd"], wl.bank)
+    got = total.cpu().numpy().astype(np.float64)
+    err = max(np.abs(got[t] - ref[t]).max() / np.abs(ref[t]).max() for t in range(T))
+    assert err <= parity.Y_TOL["bf16"], err

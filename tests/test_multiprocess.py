@@ -62,3 +62,66 @@ def test_value_is_whole_job_aggregate():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.aggregate_max(3.0, 1) == 3.0
+
+
+def test_bank_shard_partitions():
+    import sys
+    sys.path.insert(0, ROOT)
+    import predictor_gated_channel_b200 as sfn
+    for n_banks in (1, 7, 224):
+        for world in range(1, 9):
+            if world > n_banks:
+                continue
+            ranges = [sfn.bank_shard(n_banks, r, world) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == n_banks
+            assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+            sizes = [b - a for a, b in ranges]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+
+
+def _shard_worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    import predictor_gated_channel_b200 as sfn
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(5)
+        T, d, d_i, r, bank, k = 3, 16, 64, 6, 16, 4
+        x = rng.standard_normal((T, d))
+        A = rng.standard_normal((r, d)) / 4
+        B = rng.standard_normal((d_i, r)) / 2
+        Wg, Wu, Wd = (rng.standard_normal((d_i, d)) / 4 for _ in range(3))
+        b0, b1 = sfn.bank_shard(d_i // bank, rank, world)
+        rows = slice(b0 * bank, b1 * bank)
+        y_part, _, m_part = oracle.forward(x, A, B[rows], Wg[rows], Wu[rows], Wd[rows],
+                                           bank=bank, k=k)
+        t = torch.from_numpy(y_part)
+        dist.all_reduce(t)  # the collective a bank-sharded layer needs
+        y_full, _, m_full = oracle.forward(x, A, B, Wg, Wu, Wd, bank=bank, k=k)
+        out.put((rank, bool(np.allclose(t.numpy(), y_full, rtol=1e-12, atol=1e-14)),
+                 bool((m_part == m_full[:, b0:b1]).all())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bank_sharded_layer_allreduce_gloo():
+    """Two ranks hold disjoint bank ranges of one layer; their partial outputs
+    summed by an all-reduce equal the whole layer (oracle arithmetic, gloo)."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok and mask_ok for _, ok, mask_ok in res)
