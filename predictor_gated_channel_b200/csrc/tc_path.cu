@@ -70,6 +70,12 @@ struct TcParams {
   int ld_out;             // elements per output row
   int r, k, n_banks;
   bool f32_out;           // down: float32 y (no bf16 rounding), ksplit == 1
+  int a_rows;             // token rows the TMA loads per A tile (<= kBM; 0: kBM).  With
+                          // fewer tokens than a tile, rows past them are not loaded: the
+                          // MMA reads stale shared memory there, which only reaches
+                          // accumulator rows the epilogue never stores
+  uint32_t tx_bytes;      // bytes the TMA delivers per stage
+  uint32_t a_tile_bytes;  // bytes of one A tile in a stage (a_rows x 128)
   float *tau;             // top-k, if set: threshold per (token, bank) and float32 logits
                           // into out ([T][ld_out]); sig may then be null
   unsigned *err;
@@ -257,10 +263,11 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
             break;
           }
           unsigned char *a = smem + (size_t)s * p.stage_bytes;
-          unsigned char *b = a + Tr::kNumA * kTileA;
-          mbar_arrive_expect_tx(&full[s], p.stage_bytes);
+          unsigned char *b = a + Tr::kNumA * p.a_tile_bytes;
+          mbar_arrive_expect_tx(&full[s], p.tx_bytes);
           tma_load_2d(a, &tA, kb * kBK, mb * kBM, &full[s]);
-          if (Tr::kNumA == 2) tma_load_2d(a + kTileA, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
+          if (Tr::kNumA == 2)
+            tma_load_2d(a + p.a_tile_bytes, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
           if (Tr::kGateUpB) {
             tma_load_2d(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
             tma_load_2d(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
@@ -300,9 +307,9 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           }
           tc_fence_after();
           const unsigned char *a = smem + (size_t)s * p.stage_bytes;
-          const unsigned char *b = a + Tr::kNumA * kTileA;
+          const unsigned char *b = a + Tr::kNumA * p.a_tile_bytes;
           const uint64_t adesc = desc_kmajor_sw128(a);
-          const uint64_t adesc2 = desc_kmajor_sw128(a + kTileA);
+          const uint64_t adesc2 = desc_kmajor_sw128(a + p.a_tile_bytes);
           const uint64_t bdesc =
               Tr::kBMnMajor ? desc_mnmajor_sw128(b, 8192) : desc_kmajor_sw128(b);
 #pragma unroll
@@ -595,11 +602,17 @@ cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtens
                       TcParams p, int num_sms, cudaStream_t st) {
   using Tr = EpiTraits<kEpi>;
   const uint32_t b_bytes = (kEpi == kEpiDown) ? 32768u : (uint32_t)p.bn * 128u;
-  p.stage_bytes = Tr::kNumA * kTileA + b_bytes;
+  // A tiles hold only the token rows loaded; the MMA still reads kBM rows
+  // (kTileA bytes) from each A tile start, which may run past the stage: a
+  // tail of kTileA bytes keeps every such read inside the allocation
+  const uint32_t a_rows = p.a_rows > 0 ? (uint32_t)p.a_rows : (uint32_t)kBM;
+  p.a_tile_bytes = a_rows * (kBK * 2);
+  p.stage_bytes = Tr::kNumA * p.a_tile_bytes + b_bytes;
+  p.tx_bytes = p.stage_bytes;
   const size_t epi_bytes =
       (kEpi == kEpiTopk) ? (size_t)(Tr::kEpiWarps / 4) * kBM * (p.k | 1) * sizeof(float) : 0;
   // as many stages as fit beside the alignment slack, barriers and staging
-  const size_t fixed = 1024 + 256 + epi_bytes;
+  const size_t fixed = 1024 + 256 + epi_bytes + (a_rows < (uint32_t)kBM ? kTileA : 0);
   p.stages = (int)(((size_t)kMaxDynSmem - fixed) / p.stage_bytes);
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return cudaErrorInvalidValue;
@@ -645,6 +658,12 @@ TcPlan plan_tc(const FwdShape &s) {
 }
 
 namespace {
+// Token rows per A-operand TMA box: all of them when they fit one tile
+// (rounded up to 16), else a whole tile.
+int a_box_rows(const FwdShape &s) {
+  return s.T < kBM ? (int)((s.T + 15) / 16 * 16) : kBM;
+}
+
 TcParams base_params(const FwdShape &s, const DeviceInfo &dev) {
   TcParams p{};
   p.T = s.T;
@@ -654,6 +673,7 @@ TcParams base_params(const FwdShape &s, const DeviceInfo &dev) {
   p.n_banks = s.n_banks;
   p.tiles_m = (int)((s.T + kBM - 1) / kBM);
   p.ksplit = 1;
+  p.a_rows = a_box_rows(s);
   return p;
 }
 }  // namespace
@@ -679,6 +699,15 @@ static int pick_bn(int tiles_m, int n_total, std::initializer_list<int> cands, i
   return last;
 }
 
+// N tile of the logits GEMMs (the same in the forward and the backward, so
+// both see identical logits): one token tile -> two banks per tile, so that
+// both epilogue warps of a TMEM lane quadrant have a bank (measured faster
+// than one-bank tiles at 8..100 tokens); otherwise enough tiles for the SMs.
+int logits_bn(const FwdShape &s, int tiles_m, int num_sms) {
+  if (tiles_m == 1 && s.d_i % 128 == 0) return 128;
+  return pick_bn(tiles_m, s.d_i, {256, 128, 64}, num_sms);
+}
+
 int tc_h_splits(const FwdShape &s, int num_sms) {
   const int tiles = (int)((s.T + kBM - 1) / kBM) * (s.r / 64);
   const int kblocks = s.d / kBK;
@@ -697,7 +726,7 @@ cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x,
   const int bn_h = ksplit > 1 ? 64
                               : pick_bn(tiles_m, s.r, {s.r <= 256 ? s.r : s.r / 2, 64}, dev.num_sms);
   CUtensorMap mX, mA;
-  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mA, A, s.d, s.r, 64, bn_h))
+  if (!make_map(&mX, x, s.d, s.T, 64, a_box_rows(s)) || !make_map(&mA, A, s.d, s.r, 64, bn_h))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
   p.tiles_n = s.r / bn_h;
@@ -721,9 +750,10 @@ cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uin
                              cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
   const int tiles_m = (int)((s.T + kBM - 1) / kBM);
-  const int bn = pick_bn(tiles_m, s.d_i, {256, 128, 64}, dev.num_sms);
+  const int bn = logits_bn(s, tiles_m, dev.num_sms);
   CUtensorMap mH, mB;
-  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, kBM) || !make_map(&mB, B, s.r, s.d_i, 64, bn))
+  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, a_box_rows(s)) ||
+      !make_map(&mB, B, s.r, s.d_i, 64, bn))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
   p.tiles_n = s.d_i / bn;
@@ -746,9 +776,10 @@ cudaError_t launch_tc_logits_tau(const FwdShape &s, const DeviceInfo &dev, const
                                  cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
   const int tiles_m = (int)((s.T + kBM - 1) / kBM);
-  const int bn = pick_bn(tiles_m, s.d_i, {256, 128, 64}, dev.num_sms);
+  const int bn = logits_bn(s, tiles_m, dev.num_sms);
   CUtensorMap mH, mB;
-  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, kBM) || !make_map(&mB, B, s.r, s.d_i, 64, bn))
+  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, a_box_rows(s)) ||
+      !make_map(&mB, B, s.r, s.d_i, 64, bn))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
   p.tiles_n = s.d_i / bn;
@@ -776,7 +807,8 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
                           ? 128
                           : pick_bn(tiles_m, s.d_i, {128, 64}, dev.num_sms));
   CUtensorMap mX, mG, mU;
-  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mG, Wg, s.d, s.d_i, 64, bn / 2) ||
+  if (!make_map(&mX, x, s.d, s.T, 64, a_box_rows(s)) ||
+      !make_map(&mG, Wg, s.d, s.d_i, 64, bn / 2) ||
       !make_map(&mU, Wu, s.d, s.d_i, 64, bn / 2))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
@@ -799,7 +831,8 @@ cudaError_t launch_tc_dense4x_gateup(const FwdShape &s, const DeviceInfo &dev, c
   const int tiles_m = (int)((s.T + kBM - 1) / kBM);
   const int bn = 2 * pick_bn(tiles_m, s.d_i, {128, 64}, dev.num_sms);
   CUtensorMap mX, mG, mU;
-  if (!make_map(&mX, x, s.d, s.T, 64, kBM) || !make_map(&mG, Wg, s.d, s.d_i, 64, bn / 2) ||
+  if (!make_map(&mX, x, s.d, s.T, 64, a_box_rows(s)) ||
+      !make_map(&mG, Wg, s.d, s.d_i, 64, bn / 2) ||
       !make_map(&mU, Wu, s.d, s.d_i, 64, bn / 2))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
@@ -818,7 +851,8 @@ cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint1
                            const void *Wd, void *y, int ksplit, cudaStream_t st, bool f32_out) {
   if (!encoder()) return cudaErrorNotSupported;
   CUtensorMap mAct, mD;
-  if (!make_map(&mAct, act, s.d_i, s.T, 64, kBM) || !make_map(&mD, Wd, s.d, s.d_i, 64, 64))
+  if (!make_map(&mAct, act, s.d_i, s.T, 64, a_box_rows(s)) ||
+      !make_map(&mD, Wd, s.d, s.d_i, 64, 64))
     return cudaErrorInvalidValue;
   TcParams p = base_params(s, dev);
   p.tiles_n = s.d / 256;
