@@ -437,6 +437,25 @@ def run_sfn(args, rank, world, local):
         unions.append(int(bits.any(axis=0).sum()))
     union = int(round(sum(unions) / len(unions)))
 
+    # spread of the step time: R event-bracketed replays of the S-step graph
+    dist_line = None
+    if not eager:
+        R = 50 if T <= 4096 else 10
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(R)]
+        with torch.cuda.stream(stream):
+            for a, b in evs:
+                a.record(stream)
+                g_full.replay()
+                b.record(stream)
+        stream.synchronize()
+        per_step = sorted(a.elapsed_time(b) / S for a, b in evs)
+
+        def pct(q):
+            return per_step[min(R - 1, int(round(q * (R - 1))))]
+        dist_line = {"reps": R, "steps_per_rep": S, "p10_ms": pct(0.1), "p50_ms": pct(0.5),
+                     "p90_ms": pct(0.9)}
+
     # per-stage kernel times (a separate pass of eager steps, events on the stream)
     n_stage_steps = min(K, max(S, 2000 if T <= 64 else 8 * S))
     with torch.cuda.stream(stream):
@@ -580,6 +599,7 @@ def run_sfn(args, rank, world, local):
             "frac_tensor": step_flops / (elapsed_ms_max / K * 1e-3) / 1e12
                            / peaks["bf16_tflops_sustained"],
         },
+        "step_time_spread": dist_line,
         "stages": stages,
         "mask_union_channels": union,
         "cpu_baseline": cpu,

@@ -1,6 +1,8 @@
 /*
- * sfn.h -- C ABI of libsfn: the forward pass of the predictor-gated bank-wise
- * top-k sparse SwiGLU FFN on NVIDIA B200 (sm_100a).
+ * sfn.h -- C ABI of libsfn: the predictor-gated bank-wise top-k sparse
+ * SwiGLU FFN on NVIDIA B200 (sm_100a) -- its forward pass (whole layer or one
+ * bank shard), its backward with the surrogate top-k gradient, and the
+ * pages' Dense-4x comparison.
  *
  * The method: "Continual LLM Upcycling: A Predictor-Gated Bank-Wise Sparsity
  * Training Recipe for Dense-to-Sparse LLMs" (arXiv 2606.10722).  Passages are
@@ -47,11 +49,14 @@
  * `stream` (cudaStream_t; NULL is the legacy default stream) and returns
  * without synchronising; results are ready when the stream is.  No call
  * copies between host and device.  The only allocations are the
- * stream-ordered scratch of sfn_sparse_ffn_forward (cudaMallocAsync /
- * cudaFreeAsync on `stream`); the *_ws variants take caller scratch instead.
- * Calls on different streams may run concurrently if their outputs and
- * scratch do not overlap.  Results are deterministic: a fixed reduction
- * order and no floating-point atomics, so a rerun is bit-identical.
+ * stream-ordered scratch of sfn_sparse_ffn_forward and sfn_predict
+ * (cudaMallocAsync / cudaFreeAsync on `stream`) and, on the first backward
+ * call on a device, the cuBLAS handle it creates; the other entry points
+ * take caller scratch.  Calls on different streams may run concurrently if
+ * their outputs and scratch do not overlap.  Results are deterministic: a
+ * fixed reduction order and no floating-point atomics (the backward's
+ * cuBLAS GEMMs are deterministic for a given GPU), so a rerun is
+ * bit-identical.
  *
  * Errors: every argument is checked on the host before anything is
  * enqueued; on any error status nothing is written.  T == 0 returns SFN_OK
@@ -103,8 +108,9 @@ const char *sfn_status_string(sfn_status s);
 /* ABI version of this header (incremented on any signature change). */
 int sfn_abi_version(void);
 
-/* The CUDA runtime's message for the last SFN_ERR_CUDA returned on this
- * host thread (static string; "no error" if there was none). */
+/* The message behind the last SFN_ERR_CUDA (the CUDA runtime's) or the last
+ * SFN_ERR_UNSUPPORTED of the backward (why cuBLAS could not be loaded)
+ * returned on this host thread (static string; "no error" if none). */
 const char *sfn_last_error_string(void);
 
 /* Number of kernels this library has launched in this process (all

@@ -401,7 +401,7 @@ const char *sfn_status_string(sfn_status s) {
   return "unknown sfn_status";
 }
 
-int sfn_abi_version(void) { return 1; }
+int sfn_abi_version(void) { return 2; }
 
 const char *sfn_last_error_string(void) { return t_last_error; }
 

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.sfn_abi_version() == 1
+    assert L.sfn_abi_version() == 2
     for s in range(6):
         assert L.sfn_status_string(s).decode().startswith("SFN_")
     assert b"unknown" in L.sfn_status_string(99)
