@@ -210,7 +210,7 @@ sfn_status sfn_sparse_ffn_forward_static(const void *x, const void *A, const voi
  *                       the top-k and the sigma(p) g u mask fused into their
  *                       epilogues (bf16, bank 64, d and d_i multiples of
  *                       256, r a multiple of 64 up to 512);
- *   SFN_PATH_AUTO       the tensor path from T >= 8 when the shape allows
+ *   SFN_PATH_AUTO       the tensor path from T >= 6 when the shape allows
  *                       it, the CUDA-core path otherwise.
  */
 typedef enum sfn_path {

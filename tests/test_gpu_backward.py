@@ -76,7 +76,7 @@ def _check(wl, host, dev, T, bank, k, temp):
 
 
 @pytest.mark.parametrize("T,bank,k,temp", [
-    (64, 64, 16, 1.0),   # logits on the tensor cores (the forward's choice for T >= 8)
+    (64, 64, 16, 1.0),   # logits on the tensor cores (the forward's choice for T >= 6)
     (5, 64, 16, 0.5),    # logits on the CUDA-core kernels
     (33, 16, 4, 0.3),    # bank 16: CUDA-core logits
     (20, 64, 64, 1.0),   # k = bank: no threshold, no surrogate term
