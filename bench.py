@@ -610,7 +610,7 @@ def run_sfn(args, rank, world, local):
     return line
 
 
-def cpu_baseline(wl, layer_host, x_host, budget_s=12.0, method="sfn"):
+def cpu_baseline(wl, layer_host, x_host, budget_s=15.0, method="sfn"):
     """The oracle, as it stands, on a bounded sample of the same workload."""
     import numpy as np
 
@@ -633,7 +633,9 @@ def cpu_baseline(wl, layer_host, x_host, budget_s=12.0, method="sfn"):
     t0 = time.perf_counter()
     run(x_host[:1])
     t1 = time.perf_counter() - t0
-    n = max(1, min(512, int(budget_s / max(t1, 1e-3)) * max(cores, 1) // 2))
+    # about budget_s of work: one token on one core took t1, tokens run on `cores`
+    # threads (assumed ~70 % parallel efficiency)
+    n = max(1, min(16384, int(0.7 * budget_s * max(cores, 1) / max(t1, 1e-3))))
     import torch
     reps = math.ceil(n / x_host.shape[0])
     xb = torch.cat([x_host] * reps)[:n]
