@@ -173,7 +173,8 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
   unsigned char *bs = reinterpret_cast<unsigned char *>(smem_f4);      // [bank][r] (kSmemB)
   float *hs = reinterpret_cast<float *>(bs + (kSmemB ? block_bytes : 0));  // [TT][r]
   float *ps = hs + TT * r;                                              // [TT][64]
-  uint64_t *bbar = reinterpret_cast<uint64_t *>(ps + TT * 64);
+  uint32_t *pk = reinterpret_cast<uint32_t *>(ps + TT * 64);            // [TT][64] keys
+  uint64_t *bbar = reinterpret_cast<uint64_t *>(pk + TT * 64);
   const int n_banks = d_i / bank;
   const int b = blockIdx.x % n_banks;
   const int64_t t0 = (int64_t)(blockIdx.x / n_banks) * TT;
@@ -276,16 +277,16 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
         }
       }
     }
+    // the four rows' sums at once: lanes 8q .. 8q + 7 end with row q's
+    const int q = lane >> 3;
+    const int jl = jl0 + q * kWarps;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int jl = jl0 + q * kWarps;
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        const float v = warp_sum(acc[q][t]);
-        if (lane == 0 && jl < bank) {
-          ps[t * 64 + jl] = v;
-          if (kWriteLogits && t < nt) logits[(t0 + t) * d_i + b * bank + jl] = v;
-        }
+    for (int t = 0; t < TT; ++t) {
+      const float v = warp_sum4(acc[0][t], acc[1][t], acc[2][t], acc[3][t]);
+      if ((lane & 7) == 0 && jl < bank) {
+        ps[t * 64 + jl] = v;
+        pk[t * 64 + jl] = order_key(v);
+        if (kWriteLogits && t < nt) logits[(t0 + t) * d_i + b * bank + jl] = v;
       }
     }
   }
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kThreads) k_logits_topk(
   for (int t = warp; t < nt; t += kWarps) {
     const float p0 = (lane < bank) ? ps[t * 64 + lane] : 0.f;
     const float p1 = (lane + 32 < bank) ? ps[t * 64 + lane + 32] : 0.f;
-    const uint64_t word = warp_bank_topk(order_key(p0), order_key(p1), bank, k);
+    const uint64_t word = smem_bank_topk(pk + t * 64, bank, k);
     const int64_t tg = t0 + t;
     if (mask != nullptr && lane == 0) mask[tg * n_banks + b] = word;
     int *idx_row = sel_idx + tg * d_s + b * k;
@@ -348,7 +349,7 @@ cudaError_t logits_tt(const FwdShape &s, const float *h, const void *B, float *l
                       uint64_t *mask, int *sel_idx, float *sel_sig, unsigned *err,
                       cudaStream_t st) {
   const size_t block = SB ? (size_t)s.bank * s.r * E::kBytes : 0;
-  const size_t smem = block + (size_t)TT * (s.r + 64) * sizeof(float) + 16;
+  const size_t smem = block + (size_t)TT * (s.r + 128) * sizeof(float) + 16;
   auto kern = k_logits_topk<E, TT, W, K, SB>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;

@@ -159,6 +159,53 @@ struct BitonicSort<OFF, N, 2 * N> {
   __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
 };
 
+// Warp sums of four per-lane values in six shuffles (four separate
+// reductions take twenty, each a chain of dependent shuffles).  On return the
+// eight lanes with bits 4, 3 of the lane index equal to (a, b) hold the sum of
+// value 2a + b.
+__device__ __forceinline__ float warp_sum4(float v0, float v1, float v2, float v3) {
+  const int lane = threadIdx.x & 31;
+  const bool hi16 = (lane & 16) != 0, hi8 = (lane & 8) != 0;
+  float s0 = hi16 ? v2 : v0, s1 = hi16 ? v3 : v1;
+  s0 += __shfl_xor_sync(kFull, hi16 ? v0 : v2, 16);
+  s1 += __shfl_xor_sync(kFull, hi16 ? v1 : v3, 16);
+  float r = hi8 ? s1 : s0;
+  r += __shfl_xor_sync(kFull, hi8 ? s0 : s1, 8);
+  r += __shfl_xor_sync(kFull, r, 4);
+  r += __shfl_xor_sync(kFull, r, 2);
+  r += __shfl_xor_sync(kFull, r, 1);
+  return r;
+}
+
+// The same top-k, for a bank whose order keys are in shared memory (keys[j],
+// j < bank; the array padded to 64 entries with any values, 16-byte aligned),
+// by one warp: every lane reads all keys with broadcast loads and counts the
+// ranks of its two channels itself.  A chain of warp shuffles is latency
+// bound; this has no cross-lane dependency until the two ballots.
+__device__ __forceinline__ uint64_t smem_bank_topk(const uint32_t *keys, int bank, int k) {
+  if (k >= bank) return bank >= 64 ? ~0ull : ((1ull << bank) - 1ull);
+  const int lane = threadIdx.x & 31;
+  const uint32_t key0 = keys[lane], key1 = keys[lane + 32];
+  int r0 = 0, r1 = 0;
+#pragma unroll 4
+  for (int j0 = 0; j0 < 64; j0 += 4) {
+    const uint4 q = *reinterpret_cast<const uint4 *>(keys + j0);
+    const uint32_t kj[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j0 + e;
+      const bool in = j < bank;
+      r0 += in & ((kj[e] > key0) | ((kj[e] == key0) & (j < lane)));
+      r1 += in & ((kj[e] > key1) | ((kj[e] == key1) & (j < lane + 32)));
+    }
+  }
+  const bool s0 = (lane < bank) && (r0 < k);
+  const bool s1 = (lane + 32 < bank) && (r1 < k);
+  const uint32_t lo = __ballot_sync(kFull, s0);
+  const uint32_t hi = __ballot_sync(kFull, s1);
+  return ((uint64_t)hi << 32) | lo;
+}
+
 // --------------------------------------------------------------- host side
 struct DeviceInfo {
   int device = -1;
