@@ -112,6 +112,26 @@ __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x
   }
   pdl_wait();  // x may come from earlier work on the stream
   pdl_launch_dependents();
+  if (TT == 1 && nchunk <= 32 * 16) {
+    // one token, the row in one pass: every lane loads the chunks of x that
+    // match its chunks of A straight into registers (no staging, no barrier)
+    if (m >= r) return;
+    uint4 xv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int c = lane + 32 * u;
+      xv[u] = (c < nchunk) ? ld_nc16(x + (t0 * (int64_t)d + (int64_t)c * E::kVec) * E::kBytes)
+                           : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      float a[E::kVec], xf[E::kVec];
+      E::unpack(v[u], a);
+      E::unpack(xv[u], xf);
+#pragma unroll
+      for (int e = 0; e < E::kVec; ++e) acc[0] = fmaf(a[e], xf[e], acc[0]);
+    }
+  } else {
   stage_rows<E, TT>(xs, x, t0, nt, d);
   __syncthreads();
   if (m >= r) return;
@@ -137,6 +157,7 @@ __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x
         }
       }
     }
+  }
   }
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
@@ -332,7 +353,8 @@ __global__ void __launch_bounds__(kThreads) k_bank_topk(const float *__restrict_
 template <class E, int TT, bool SPLIT>
 cudaError_t pred_h_tt(const FwdShape &s, const void *x, const void *A, void *h,
                       const void *pf, size_t pf_bytes, cudaStream_t st) {
-  const size_t smem = (size_t)TT * s.d * sizeof(float);
+  // one token: x goes straight to registers, no staging
+  const size_t smem = (TT == 1 && s.d / E::kVec <= 32 * 16) ? 0 : (size_t)TT * s.d * sizeof(float);
   auto kern = k_pred_h<E, TT, SPLIT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
