@@ -355,7 +355,7 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
       e = timed(SFN_STAGE_REDUCE, st,
                 [&] {
                   return launch_reduce_partials(s, p.cpt, partial, y, st,
-                                                y_f32 ? ReduceOut::kYF32 : ReduceOut::kYLast);
+                                                y_f32 ? ReduceOut::kYF32 : ReduceOut::kY);
                 });
   }
   if (own_ws) {

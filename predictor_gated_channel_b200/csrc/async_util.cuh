@@ -111,6 +111,13 @@ __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// Hint: bring the line holding p into L2 through this thread's own load
+// path (also fills the address translation that later loads of the line
+// use).  Any address of mapped memory; the line may still be being written.
+__device__ __forceinline__ void prefetch_line_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Programmatic dependent launch: let the next kernel in the stream start its
 // prologue now / wait until the previous kernel has completed and its memory
 // is visible.  Both are no-ops when the launch carries no such dependency.

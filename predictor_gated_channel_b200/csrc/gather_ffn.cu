@@ -228,44 +228,67 @@ __global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
 
 // out[t][c0 .. c0+C) = sum_{c < cpt} partial[t][c][c0 .. c0+C), summed in a
 // fixed order.  blockIdx.x = t * ceil(n / C) + slice.  Thread = (group g,
-// quad q): group g sums partials c = g, g + G, ...; the G group sums are then
-// added in group order.  kOut: 0 = float32 out, 1 = bf16 out, 2 = bf16 hi/lo
-// halves of h ([T][2n]: hi at column j, lo = bf16(sum - hi) at n + j).
-template <int C, int kOut, bool kEarly>
+// quad q), q fastest: group g sums partials c = g, g + G, ... (its loads
+// issued as one batch of kBatch); the four groups of a warp that share q are
+// combined by two shuffles, then the warps' sums in warp order.  kOut: 0 =
+// float32 out, 1 = bf16 out, 2 = bf16 hi/lo halves of h ([T][2n]: hi at
+// column j, lo = bf16(sum - hi) at n + j).
+template <int C, int kOut>
 __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
     const float *__restrict__ partial, void *__restrict__ out, int n, int cpt) {
   constexpr int Q = C / 4;                // float4 quads per slice
   constexpr int G = kReduceThreads / Q;   // partial groups
-  __shared__ float4 red[G][Q];
+  constexpr int kWarps = kReduceThreads / 32;
+  constexpr int kBatch = 8;               // loads per thread in flight
+  static_assert(Q == 8 || Q == 32, "a warp holds 4 groups of 8 quads or 1 group of 32");
+  __shared__ float4 red[kWarps][Q];
   const int slices = (n + C - 1) / C;
   const int64_t t = blockIdx.x / slices;
   const int c0 = (blockIdx.x % slices) * C;
   const int g = threadIdx.x / Q, q = threadIdx.x % Q;
   const int col = c0 + q * 4;
-  // kEarly (last kernel of a forward call): the next call's first kernel may
-  // start at once; it reads only weights before its own griddepcontrol.wait,
-  // which returns after this kernel -- and so everything before it -- is done
-  if (kEarly) pdl_launch_dependents();
+  // The stream's next kernel is released once the partials are complete, not
+  // earlier: the next forward call's first kernel prefetches the predictor's
+  // B into L2, which is cheaper here, with DRAM otherwise idle, than during
+  // the bandwidth-bound gate/up/down kernel.
   pdl_wait();
-  if (!kEarly) pdl_launch_dependents();
+  pdl_launch_dependents();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (col < n) {
     const float *p = partial + t * cpt * (int64_t)n + col;
-#pragma unroll 8
-    for (int c = g; c < cpt; c += G) {
-      const float4 v = *reinterpret_cast<const float4 *>(p + (int64_t)c * n);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+    for (int cb = g; cb < cpt; cb += kBatch * G) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        v[u] = (cb + u * G < cpt) ? *reinterpret_cast<const float4 *>(p + (int64_t)(cb + u * G) * n)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        acc.x += v[u].x;
+        acc.y += v[u].y;
+        acc.z += v[u].z;
+        acc.w += v[u].w;
+      }
     }
   }
-  red[g][q] = acc;
+  // lanes q, q + 8, q + 16, q + 24 of a warp hold groups of the same quad
+  if (Q == 8) {
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) {
+      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane < Q) red[warp][lane] = acc;
   __syncthreads();
   if (threadIdx.x < Q) {
     float4 v = red[0][threadIdx.x];
-    for (int gg = 1; gg < G; ++gg) {
-      const float4 r4 = red[gg][threadIdx.x];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      const float4 r4 = red[w][threadIdx.x];
       v.x += r4.x;
       v.y += r4.y;
       v.z += r4.z;
@@ -347,17 +370,10 @@ cudaError_t reduce_c(const FwdShape &s, int n, int cpt, const float *partial, vo
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const dim3 grid((unsigned)blocks), block(kReduceThreads);
   if (kind == ReduceOut::kSplitH)
-    return launch_pdl(k_reduce_partials<C, 2, false>, grid, block, 0, st, partial, out, n, cpt);
-  if (kind == ReduceOut::kYF32)
-    return launch_pdl(k_reduce_partials<C, 0, false>, grid, block, 0, st, partial, out, n, cpt);
-  if (kind == ReduceOut::kYLast) {
-    if (s.bf16)
-      return launch_pdl(k_reduce_partials<C, 1, true>, grid, block, 0, st, partial, out, n, cpt);
-    return launch_pdl(k_reduce_partials<C, 0, true>, grid, block, 0, st, partial, out, n, cpt);
-  }
-  if (s.bf16)
-    return launch_pdl(k_reduce_partials<C, 1, false>, grid, block, 0, st, partial, out, n, cpt);
-  return launch_pdl(k_reduce_partials<C, 0, false>, grid, block, 0, st, partial, out, n, cpt);
+    return launch_pdl(k_reduce_partials<C, 2>, grid, block, 0, st, partial, out, n, cpt);
+  if (kind == ReduceOut::kY && s.bf16)
+    return launch_pdl(k_reduce_partials<C, 1>, grid, block, 0, st, partial, out, n, cpt);
+  return launch_pdl(k_reduce_partials<C, 0>, grid, block, 0, st, partial, out, n, cpt);
 }
 
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,

@@ -110,6 +110,13 @@ __global__ void __launch_bounds__(kThreadsH) k_pred_h(const char *__restrict__ x
     const int c = lane + 32 * u;
     v[u] = (m < r && c < nchunk) ? ld_stream16(row + (int64_t)c * 16) : make_uint4(0, 0, 0, 0);
   }
+  // x's lines: warm before the wait (a hint; the loads below come after it)
+  {
+    const int64_t xb = (int64_t)nt * d * E::kBytes;
+    const char *xr = x + t0 * (int64_t)d * E::kBytes;
+    for (int64_t o = (int64_t)threadIdx.x * 128; o < xb; o += (int64_t)blockDim.x * 128)
+      prefetch_line_l2(xr + o);
+  }
   pdl_wait();  // x may come from earlier work on the stream
   pdl_launch_dependents();
   if (TT == 1 && nchunk <= 32 * 16) {

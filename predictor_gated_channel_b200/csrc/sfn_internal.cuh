@@ -284,12 +284,10 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
                        const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
                        float *partial, unsigned *err, cudaStream_t st);
 // Output of k_reduce_partials: y in the call's element type, or the bf16
-// hi/lo halves of h ([T][2r], "split").  kYLast: y, from the last kernel of
-// a call on the CUDA-core path, which lets the stream's next kernel start
-// its (weights-only) prologue at once.
+// hi/lo halves of h ([T][2r], "split").
 // kYF32: y as float32 whatever the input type (partial outputs of a bank
 // shard, summed across devices before rounding).
-enum class ReduceOut { kY, kYLast, kYF32, kSplitH };
+enum class ReduceOut { kY, kYF32, kSplitH };
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
                                    cudaStream_t st, ReduceOut kind = ReduceOut::kY);
 
