@@ -244,6 +244,35 @@ def test_tensor_path_k_variants(k, full_layer):
     _check_forward(host, x, y, mask, 64, k, "bf16", rows=rows)
 
 
+@pytest.mark.parametrize("k", [1, 4, 16, 20])
+def test_tensor_topk_exact_ties(k):
+    """One-hot tokens and small-integer A and B make the tensor-core logits
+    exact integers; every bank of B holds 16 rows four times each, so exact
+    ties are everywhere.  The mask of the top-k fused into the logits GEMM
+    equals the oracle's bit for bit (ties to the lower channel), for k below
+    16, at 16 and above 16 (the wider-staging variant)."""
+    rng = np.random.default_rng(300 + k)
+    T, d, d_i, r = 130, 256, 1024, 64
+    x = np.zeros((T, d), np.float32)
+    x[np.arange(T), rng.integers(0, d, T)] = 1.0
+    A = rng.integers(-3, 4, (r, d)).astype(np.float32)
+    B = rng.integers(-2, 3, (d_i, r)).astype(np.float32)
+    for b in range(d_i // 64):
+        B[b * 64:(b + 1) * 64] = np.tile(B[b * 64:b * 64 + 16], (4, 1))[rng.permutation(64)]
+    W = (rng.standard_normal((d_i, d)) * 0.05).astype(np.float32)
+
+    def dev_bf16(a):
+        return torch.from_numpy(a).to(torch.bfloat16).to(DEV)
+
+    _, mask = sfn.sparse_ffn_forward(dev_bf16(x), dev_bf16(A), dev_bf16(B), dev_bf16(W),
+                                     dev_bf16(W), dev_bf16(W), bank=64, k=k, path="tensor")
+    torch.cuda.synchronize()
+    p = (x.astype(np.int64) @ A.T.astype(np.int64)) @ B.T.astype(np.int64)
+    assert np.abs(p).max() < 2 ** 24  # exact in float32
+    want = oracle.bank_topk(p.astype(np.float32), 64, k)
+    assert np.array_equal(parity.to_u64(mask), want)
+
+
 def test_paths_agree(full_layer):
     """CUDA-core and tensor paths on the same 96 tokens: masks differ only at
     allowed near-ties, outputs within the bf16 tolerance of each other."""
