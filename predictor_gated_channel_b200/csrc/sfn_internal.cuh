@@ -124,12 +124,14 @@ __device__ __forceinline__ void cex_desc(uint32_t &a, uint32_t &b) {
   b = lo;
 }
 
-// Bitonic network sorting s[OFF, OFF + N) in descending order.  Every index
-// is a compile-time constant (the stages are template-recursive), so the
-// array stays in registers.
+// Bitonic network sorting s[OFF, OFF + N) of an array of any length in
+// descending order.  Every index is a compile-time constant (the stages are
+// template-recursive), so the array stays in registers.
 template <int OFF, int N, int SIZE, int STRIDE>
 struct BitonicStage {
-  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
+  template <int L>
+  __device__ __forceinline__ static void run(uint32_t (&s)[L]) {
+    static_assert(OFF + N <= L, "network outside the array");
 #pragma unroll
     for (int i = 0; i < N; ++i) {
       const int j = i ^ STRIDE;
@@ -145,18 +147,21 @@ struct BitonicStage {
 };
 template <int OFF, int N, int SIZE>
 struct BitonicStage<OFF, N, SIZE, 0> {
-  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
+  template <int L>
+  __device__ __forceinline__ static void run(uint32_t (&)[L]) {}
 };
 template <int OFF, int N, int SIZE>
 struct BitonicSort {
-  __device__ __forceinline__ static void run(uint32_t (&s)[64]) {
+  template <int L>
+  __device__ __forceinline__ static void run(uint32_t (&s)[L]) {
     BitonicStage<OFF, N, SIZE, SIZE / 2>::run(s);
     BitonicSort<OFF, N, SIZE * 2>::run(s);
   }
 };
 template <int OFF, int N>
 struct BitonicSort<OFF, N, 2 * N> {
-  __device__ __forceinline__ static void run(uint32_t (&)[64]) {}
+  template <int L>
+  __device__ __forceinline__ static void run(uint32_t (&)[L]) {}
 };
 
 // Warp sums of four per-lane values in six shuffles (four separate

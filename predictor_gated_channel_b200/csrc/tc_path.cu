@@ -173,34 +173,52 @@ __device__ __forceinline__ void bank_threshold(uint32_t taddr, int k, uint32_t &
     gt = 0;
     return;
   }
+  if (k <= 16) {
+    // A running list of the 16 largest keys, sorted descending, merged with
+    // each sorted group of 16 in turn.  A loop, not unrolled: the straight-line
+    // version of this epilogue was long enough to stall on instruction fetch.
+    // Keys are >= 0, so starting from zeros the first merge takes group 0 as is.
+    uint32_t top[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) top[i] = 0u;
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(taddr + g * 16, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) r[i] = order_key(__uint_as_float(r[i]));
+      BitonicSort<0, 16, 2>::run(r);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) top[i] = max(top[i], r[15 - i]);
+#pragma unroll
+      for (int stride = 8; stride > 0; stride >>= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if ((i & stride) == 0) cex_desc(top[i], top[i + stride]);
+    }
+    tau = top[0];
+#pragma unroll
+    for (int i = 1; i < 16; ++i) tau = (i == k - 1) ? top[i] : tau;
+    gt = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) gt += top[i] > tau;
+    return;
+  }
+  // k > 16: sort all 64 keys
   uint32_t s[64];
   tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
   tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
   tmem_ld_wait();
 #pragma unroll
   for (int i = 0; i < 64; ++i) s[i] = order_key(__uint_as_float(s[i]));
+  BitonicSort<0, 64, 2>::run(s);
+  tau = s[0];
+#pragma unroll
+  for (int i = 1; i < 64; ++i) tau = (i == k - 1) ? s[i] : tau;
   gt = 0;
-  if (k == 16) {
-    BitonicSort<0, 16, 2>::run(s);
-    BitonicSort<16, 16, 2>::run(s);
-    BitonicSort<32, 16, 2>::run(s);
-    BitonicSort<48, 16, 2>::run(s);
-    merge_top16<0, 16>(s);
-    merge_top16<32, 48>(s);
-    // the 16 largest overall: max(s[i], s[47 - i]), i < 16
-    tau = 0xffffffffu;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) tau = min(tau, max(s[i], s[47 - i]));
-#pragma unroll
-    for (int i = 0; i < 16; ++i) gt += max(s[i], s[47 - i]) > tau;
-  } else {
-    BitonicSort<0, 64, 2>::run(s);
-    tau = s[0];
-#pragma unroll
-    for (int i = 1; i < 64; ++i) tau = (i == k - 1) ? s[i] : tau;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) gt += s[i] > tau;
-  }
+  for (int i = 0; i < 64; ++i) gt += s[i] > tau;
 }
 
 template <int kEpi>
@@ -413,22 +431,24 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           const int need = p.k - gt;
           const int bank = nb * banks_per_tile + bl;
           int eq = 0, cnt = 0;
-          uint32_t bits[2], rest = 0u;  // rest: largest key not kept
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(taddr + bl * 64 + half * 32, v);
+          uint64_t word = 0ull;
+          uint32_t rest = 0u;  // rest: largest key not kept
+          // four groups of 16 channels, as a loop (code size, as above)
+#pragma unroll 1
+          for (int g = 0; g < 4; ++g) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(taddr + bl * 64 + g * 16, v);
             tmem_ld_wait();
             if (p.tau != nullptr && valid) {
               uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<float *>(p.out) +
-                                                     t * p.ld_out + bank * 64 + half * 32);
+                                                     t * p.ld_out + bank * 64 + g * 16);
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
+              for (int i = 0; i < 4; ++i)
                 dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
             uint32_t b = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 16; ++i) {
               const uint32_t key = order_key(__uint_as_float(v[i]));
               const bool take = (key > tau) | ((key == tau) & (eq < need));
               eq += (key == tau);
@@ -437,13 +457,13 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
               if (take) stg[cnt] = __uint_as_float(v[i]);
               cnt += take;
             }
-            bits[half] = b;
+            word |= (uint64_t)b << (g * 16);
           }
           if (valid && p.tau != nullptr)
             p.tau[t * p.n_banks + bank] = (p.k < 64)
                                               ? 0.5f * (key_value(tau) + key_value(rest))
                                               : __int_as_float(0x7fc00000);
-          if (valid) p.mask[t * p.n_banks + bank] = ((uint64_t)bits[1] << 32) | bits[0];
+          if (valid) p.mask[t * p.n_banks + bank] = word;
           if (valid && p.sig != nullptr) {
             float *sig_out = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
             if ((p.k & 3) == 0) {
