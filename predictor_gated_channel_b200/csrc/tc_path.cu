@@ -78,6 +78,8 @@ struct TcParams {
   uint32_t a_tile_bytes;  // bytes of one A tile in a stage (a_rows x 128)
   float *tau;             // top-k, if set: threshold per (token, bank) and float32 logits
                           // into out ([T][ld_out]); sig may then be null
+  bool b_once;            // the B operand (weights) is read once (one token tile): its
+                          // loads carry an evict-first L2 policy
   unsigned *err;
 };
 
@@ -270,6 +272,13 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
       if (Tr::kGateUpB) prefetch_tmap(&tB2);
       uint32_t it = 0;
       bool ok = true;
+      const uint64_t once = make_evict_first_policy();
+      auto load_b = [&](void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+        if (p.b_once)
+          tma_load_2d_hint(dst, map, c0, c1, bar, once);
+        else
+          tma_load_2d(dst, map, c0, c1, bar);
+      };
       for (int unit = blockIdx.x; unit < total && ok; unit += gridDim.x) {
         int mb, nb, kb0, kb1;
         unit_coords(unit, p, mb, nb, kb0, kb1);
@@ -287,14 +296,14 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           if (Tr::kNumA == 2)
             tma_load_2d(a + p.a_tile_bytes, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
           if (Tr::kGateUpB) {
-            tma_load_2d(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
-            tma_load_2d(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
+            load_b(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
+            load_b(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
           } else if (kEpi == kEpiDown) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              tma_load_2d(b + q * 8192, &tB, nb * kAccCols + q * 64, kb * kBK, &full[s]);
+              load_b(b + q * 8192, &tB, nb * kAccCols + q * 64, kb * kBK, &full[s]);
           } else {
-            tma_load_2d(b, &tB, kb * kBK, nb * p.bn, &full[s]);
+            load_b(b, &tB, kb * kBK, nb * p.bn, &full[s]);
           }
         }
       }
@@ -694,6 +703,7 @@ TcParams base_params(const FwdShape &s, const DeviceInfo &dev) {
   p.tiles_m = (int)((s.T + kBM - 1) / kBM);
   p.ksplit = 1;
   p.a_rows = a_box_rows(s);
+  p.b_once = (p.tiles_m == 1);
   return p;
 }
 }  // namespace
