@@ -89,8 +89,11 @@ struct EpiTraits {
   static constexpr bool kBMnMajor = (kEpi == kEpiDown);
   static constexpr bool kGateUpB = (kEpi == kEpiGateUp || kEpi == kEpiDense4x);
   // epilogue warps: two per TMEM lane quadrant for the top-k (its sorting
-  // networks, not the MMAs, bound that GEMM), splitting the tile's banks
-  static constexpr int kEpiWarps = (kEpi == kEpiTopk) ? 8 : 4;
+  // networks, not the MMAs, bound that GEMM) and for gate/up and down (with
+  // one tile per CTA at few tokens, their epilogue is a serial tail after
+  // the mainloop), splitting the tile's banks or column chunks
+  static constexpr int kEpiWarps =
+      (kEpi == kEpiTopk || kEpi == kEpiGateUp || kEpi == kEpiDown) ? 8 : 4;
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
 };
 
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           }
         }
       } else if (kEpi == kEpiLogits || kEpi == kEpiDown || kEpi == kEpiHSplit) {
-        for (int c0 = 0; c0 < p.bn; c0 += 32) {
+        for (int c0 = 32 * half_id; c0 < p.bn; c0 += 32 * (Tr::kEpiWarps / 4)) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + c0, v);
           tmem_ld_wait();
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
         // [0, bn/2) hold g, [bn/2, bn) hold u
         uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
         const int half_n = p.bn / 2;
-        for (int h = 0; h < half_n / 64; ++h) {
+        for (int h = half_id; h < half_n / 64; h += Tr::kEpiWarps / 4) {
           const int bank = nb * (half_n / 64) + h;
           const uint64_t word = valid ? p.mask[t * p.n_banks + bank] : 0ull;
           const float *sig_in = p.sig + (t * p.n_banks + bank) * (int64_t)p.k;
