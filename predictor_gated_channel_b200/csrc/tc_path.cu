@@ -264,8 +264,14 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // operands may come from earlier work on the stream
-  pdl_launch_dependents();
+  // Operands may come from earlier work on the stream.  The producer waits
+  // later: the weights (every GEMM's B operand) are not written by earlier
+  // work, so with one token tile it issues the first stages' weight loads
+  // before its wait.
+  if (!p.b_once || warp != 0) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -282,6 +288,36 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
         else
           tma_load_2d(dst, map, c0, c1, bar);
       };
+      // the weights of stage s for K block kb and N tile nb
+      auto issue_b = [&](int s, int kb, int nb) {
+        unsigned char *b = smem + (size_t)s * p.stage_bytes + Tr::kNumA * p.a_tile_bytes;
+        if (Tr::kGateUpB) {
+          load_b(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
+          load_b(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
+        } else if (kEpi == kEpiDown) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            load_b(b + q * 8192, &tB, nb * kAccCols + q * 64, kb * kBK, &full[s]);
+        } else {
+          load_b(b, &tB, kb * kBK, nb * p.bn, &full[s]);
+        }
+      };
+      // before the wait (one token tile only): the weights of the first
+      // unit's first stages
+      int pre = 0;
+      if (p.b_once && (int)blockIdx.x < total) {
+        int mb, nb, kb0, kb1;
+        unit_coords(blockIdx.x, p, mb, nb, kb0, kb1);
+        pre = min(p.stages, kb1 - kb0);
+        for (int j = 0; j < pre; ++j) {
+          mbar_arrive_expect_tx(&full[j], p.tx_bytes);
+          issue_b(j, kb0 + j, nb);
+        }
+      }
+      if (p.b_once) {
+        pdl_wait();
+        pdl_launch_dependents();
+      }
       for (int unit = blockIdx.x; unit < total && ok; unit += gridDim.x) {
         int mb, nb, kb0, kb1;
         unit_coords(unit, p, mb, nb, kb0, kb1);
@@ -293,29 +329,23 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
             break;
           }
           unsigned char *a = smem + (size_t)s * p.stage_bytes;
-          unsigned char *b = a + Tr::kNumA * p.a_tile_bytes;
-          mbar_arrive_expect_tx(&full[s], p.tx_bytes);
+          if ((int)it >= pre) mbar_arrive_expect_tx(&full[s], p.tx_bytes);
           tma_load_2d(a, &tA, kb * kBK, mb * kBM, &full[s]);
           if (Tr::kNumA == 2)
             tma_load_2d(a + p.a_tile_bytes, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
-          if (Tr::kGateUpB) {
-            load_b(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
-            load_b(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
-          } else if (kEpi == kEpiDown) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              load_b(b + q * 8192, &tB, nb * kAccCols + q * 64, kb * kBK, &full[s]);
-          } else {
-            load_b(b, &tB, kb * kBK, nb * p.bn, &full[s]);
-          }
+          if ((int)it >= pre) issue_b(s, kb, nb);
         }
       }
-      // wait (bounded) until the last load of every stage has landed
-      const uint32_t issued = it;
+      // wait (bounded) until the last load of every stage has landed (a
+      // stage whose weights went out before the wait counts as issued)
+      const uint32_t issued = it > (uint32_t)pre ? it : (uint32_t)pre;
       for (int s = 0; s < p.stages && (uint32_t)s < issued; ++s) {
         const uint32_t last = s + ((issued - 1 - s) / p.stages) * p.stages;
         mbar_wait(&full[s], (last / p.stages) & 1u, p.err);
       }
+    } else if (p.b_once) {
+      pdl_wait();
+      pdl_launch_dependents();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
