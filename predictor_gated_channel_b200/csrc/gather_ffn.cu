@@ -321,6 +321,67 @@ __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
   }
 }
 
+// Four consecutive outputs v at out[i .. i + 4): kOut 0 float32, 1 bf16.
+template <int kOut>
+__device__ __forceinline__ void store_quad(void *out, int64_t i, float4 v) {
+  if (kOut == 0) {
+    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + i) = v;
+  } else {
+    uint2 o;
+    o.x = (uint32_t)f32_to_bf16_bits(v.x) | ((uint32_t)f32_to_bf16_bits(v.y) << 16);
+    o.y = (uint32_t)f32_to_bf16_bits(v.z) | ((uint32_t)f32_to_bf16_bits(v.w) << 16);
+    *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(out) + i) = o;
+  }
+}
+
+// Few partials (cpt <= kSmallCpt): one thread per four columns adds the cpt
+// partial rows in order 0, 1, ..., with its loads in flight together.  No
+// shared memory, so its CTAs fit beside a large-shared-memory kernel still
+// running on the SM and start early (programmatic dependent launch).
+constexpr int kSmallCpt = 16;
+template <int kOut>
+__global__ void __launch_bounds__(kReduceThreads) k_reduce_few(
+    const float *__restrict__ partial, void *__restrict__ out, int n, int cpt) {
+  const int per_t = (n / 4 + kReduceThreads - 1) / kReduceThreads;
+  const int64_t t = blockIdx.x / per_t;
+  const int col = ((blockIdx.x % per_t) * kReduceThreads + threadIdx.x) * 4;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (col >= n) return;
+  const float *p = partial + t * cpt * (int64_t)n + col;
+  float4 v[kSmallCpt];
+#pragma unroll
+  for (int c = 0; c < kSmallCpt; ++c)
+    v[c] = (c < cpt) ? *reinterpret_cast<const float4 *>(p + (int64_t)c * n)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 acc = v[0];
+#pragma unroll
+  for (int c = 1; c < kSmallCpt; ++c) {
+    if (c < cpt) {
+      acc.x += v[c].x;
+      acc.y += v[c].y;
+      acc.z += v[c].z;
+      acc.w += v[c].w;
+    }
+  }
+  if (kOut == 0 || kOut == 1) {
+    store_quad<kOut == 0 ? 0 : 1>(out, t * n + col, acc);
+  } else {
+    const float f[4] = {acc.x, acc.y, acc.z, acc.w};
+    uint16_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      hi[e] = f32_to_bf16_bits(f[e]);
+      lo[e] = f32_to_bf16_bits(f[e] - __uint_as_float((uint32_t)hi[e] << 16));
+    }
+    uint16_t *h2 = reinterpret_cast<uint16_t *>(out) + t * 2 * n;
+    *reinterpret_cast<uint2 *>(h2 + col) =
+        make_uint2(hi[0] | ((uint32_t)hi[1] << 16), hi[2] | ((uint32_t)hi[3] << 16));
+    *reinterpret_cast<uint2 *>(h2 + n + col) =
+        make_uint2(lo[0] | ((uint32_t)lo[1] << 16), lo[2] | ((uint32_t)lo[3] << 16));
+  }
+}
+
 template <class E>
 cudaError_t ffn_e(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
                   const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
@@ -379,9 +440,23 @@ cudaError_t reduce_c(const FwdShape &s, int n, int cpt, const float *partial, vo
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
                                    cudaStream_t st, ReduceOut kind) {
   const int n = (kind == ReduceOut::kSplitH) ? s.r : s.d;
-  // many partials: narrow slices and 32 partial groups; few: wide slices
-  cudaError_t e = cpt >= 32 ? reduce_c<32>(s, n, cpt, partial, y, kind, st)
-                            : reduce_c<128>(s, n, cpt, partial, y, kind, st);
+  cudaError_t e;
+  if (cpt <= kSmallCpt && n % 4 == 0) {
+    const int per_t = (n / 4 + kReduceThreads - 1) / kReduceThreads;
+    const int64_t blocks = (int64_t)per_t * s.T;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const dim3 grid((unsigned)blocks), block(kReduceThreads);
+    if (kind == ReduceOut::kSplitH)
+      e = launch_pdl(k_reduce_few<2>, grid, block, 0, st, partial, y, n, cpt);
+    else if (kind == ReduceOut::kY && s.bf16)
+      e = launch_pdl(k_reduce_few<1>, grid, block, 0, st, partial, y, n, cpt);
+    else
+      e = launch_pdl(k_reduce_few<0>, grid, block, 0, st, partial, y, n, cpt);
+  } else {
+    // many partials: narrow slices and 32 partial groups; else wide slices
+    e = cpt >= 32 ? reduce_c<32>(s, n, cpt, partial, y, kind, st)
+                  : reduce_c<128>(s, n, cpt, partial, y, kind, st);
+  }
   count_launches(1);
   return e;
 }
