@@ -222,7 +222,7 @@ def test_zero_tokens(full_layer):
 
 # ------------------------------------------------------------------ tensor path
 
-@pytest.mark.parametrize("T", [1, 5, 128, 130, 300])
+@pytest.mark.parametrize("T", [1, 5, 64, 128, 130, 300])
 def test_tensor_path_full_width(T, full_layer):
     """The tcgen05 path (forced) against the oracle, every token checked."""
     wl, host, dev = full_layer
