@@ -78,14 +78,6 @@ int pow2_tokens(int64_t T, int cap) {
 
 void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
-bool debug_enabled() {
-  static const bool on = [] {
-    const char *v = getenv("SFN_DEBUG");
-    return v != nullptr && v[0] == '1';
-  }();
-  return on;
-}
-
 cudaError_t ensure_smem_limit(const void *kernel, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   int dev = 0;

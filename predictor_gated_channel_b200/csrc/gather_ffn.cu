@@ -16,8 +16,11 @@
 //                      down warp owns one eighth of the output columns in
 //                      registers and accumulates a * Wd[j, cols] over the
 //                      slots in order.  The CTA writes one fp32 partial row.
-//   k_reduce_partials  y[t] = sum of the token's partial rows in CTA order,
-//                      rounded to the output type.
+//   k_reduce_partials  y[t] = sum of the token's partial rows in a fixed
+//                      order, rounded to the output type.  Also the tensor
+//                      path's split-K sums (fp32 partials of h and of y).
+//   k_reduce_few       the same for at most 16 partials: one thread per four
+//                      columns, no shared memory.
 // Only the kept rows of Wg, Wu and Wd are read, each once per token; all sums
 // run in a fixed order, so results are bit-reproducible.
 #include "async_util.cuh"
@@ -248,9 +251,9 @@ __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
   const int g = threadIdx.x / Q, q = threadIdx.x % Q;
   const int col = c0 + q * 4;
   // The stream's next kernel is released once the partials are complete, not
-  // earlier: the next forward call's first kernel prefetches the predictor's
-  // B into L2, which is cheaper here, with DRAM otherwise idle, than during
-  // the bandwidth-bound gate/up/down kernel.
+  // earlier.  As the last kernel of a CUDA-core forward call, this puts the
+  // next call's prologue (its L2 prefetch of the predictor's B) in DRAM's
+  // idle time here rather than in the bandwidth-bound gate/up/down kernel.
   pdl_wait();
   pdl_launch_dependents();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -223,9 +223,6 @@ bool device_info(DeviceInfo *out);
 
 void count_launches(uint64_t n);
 
-// SFN_DEBUG=1 in the environment: diagnostic messages on stderr.
-bool debug_enabled();
-
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
