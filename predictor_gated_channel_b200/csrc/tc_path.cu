@@ -23,9 +23,14 @@
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
 //               (M 128, N <= 256, K 16, bf16 -> f32) into one of two TMEM
 //               accumulators and commits stage releases / tile completions
-//   warps 2..5  epilogue: tcgen05.ld of the warp's 32 TMEM lanes (= 32 token
-//               rows), the epilogue arithmetic, global stores; they release
-//               the accumulator so the next tile's MMAs overlap this epilogue
+//   warps 2..   epilogue (4 warps for G1, 8 for G2-G4: two per TMEM lane
+//               quadrant, splitting a tile's banks or column chunks):
+//               tcgen05.ld of the warp's 32 TMEM lanes (= 32 token rows), the
+//               epilogue arithmetic, global stores; they release the
+//               accumulator so the next tile's MMAs overlap this epilogue
+// With one token tile every weight byte is read once: the weight loads then
+// carry an evict-first L2 policy, and the producer issues the first stages'
+// weight loads before its dependency wait.
 // Every mbarrier wait is bounded (async_util.cuh).
 #include <cudaTypedefs.h>
 
