@@ -7,7 +7,8 @@
 //
 //   k_pred_h       h[t] = A x[t] (fp32), one warp per row of A with the whole
 //                  row's 16-byte loads in flight; token groups of TT share
-//                  each row load.
+//                  each row load.  x's lines are L2-prefetched before the
+//                  wait; one token's x then goes straight into registers.
 //   k_logits_topk  p[t] = B h[t] for one bank, then (optionally) that bank's
 //                  top-k: mask word, kept channel ids and sigma(p) in
 //                  ascending channel order (one CTA per bank and token group).
@@ -18,7 +19,8 @@
 // The chained kernels use programmatic dependent launch.  Each calls
 // griddepcontrol.wait before touching anything an earlier kernel writes and
 // only then lets its dependent start, so a dependent's prologue (which reads
-// nothing but weights) always runs after all work before its predecessor.
+// nothing but weights; the L2 prefetch of x is a hint, not a read of its
+// values) always runs after all work before its predecessor.
 #include "async_util.cuh"
 #include "sfn_internal.cuh"
 
