@@ -241,8 +241,9 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
 // The CUDA-core path streams each token's kept rows separately (T x 88 MB for
 // the 4096 x 14336 layer), bound by what each SM can pull; the tensor path
 // reads the union of the tokens' kept rows once, with dense tiles.  Measured
-// graph-replayed step times on that layer (bf16, B200): T = 4: 71 vs 98 us;
-// T = 6: 100 vs 99 us; T = 8: 118 vs 100 us.
+// graph-replayed step times on that layer (bf16, B200), CUDA-core vs tensor:
+// T = 4: 67 vs 86 us; T = 5: 86 vs 87 us; T = 6: 96 vs 87 us; T = 8: 114 vs
+// 87 us.
 constexpr int64_t kTcMinTokens = 6;
 bool use_tensor_path(const FwdShape &s, sfn_path path) {
   if (path == SFN_PATH_CUDA_CORE) return false;
