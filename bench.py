@@ -64,6 +64,10 @@ def parse_args(argv=None):
                     help="surrogate temperature of --method backward")
     ap.add_argument("--path", default="auto", choices=["auto", "cuda_core", "tensor"],
                     help="kernels to use (the library picks by token count when auto)")
+    ap.add_argument("--workloads", default="all", choices=["all", "one"],
+                    help="all (default): with the default decode workload, also measure the "
+                         "batched-decode, prefill and long-prefill workloads and report them "
+                         "under 'workloads'; one: only --workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--settle", type=float, default=1.0,
@@ -92,8 +96,11 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def default_steps(name):
-    # about a second of timed GPU work at the current kernel speeds
+def default_steps(name, extra=False):
+    # about a second of timed GPU work at the current kernel speeds; the
+    # workloads measured beside the headline line take about a quarter second
+    if extra:
+        return {"decode": 10000, "batched_decode": 2000, "prefill": 100, "long_prefill": 20}[name]
     return {"decode": 40000, "batched_decode": 4000, "prefill": 200, "long_prefill": 30}[name]
 
 
@@ -253,14 +260,10 @@ def useful_flops_per_token(wl, method="sfn"):
 # ---------------------------------------------------------------------- the GPU arm
 
 def run_sfn(args, rank, world, local):
-    import numpy as np
     import torch
 
-    import predictor_gated_channel_b200 as sfn
     from predictor_gated_channel_b200 import _capi
     from predictor_gated_channel_b200 import build as sfn_build
-    from predictor_gated_channel_b200.inputs import (WORKLOADS, make_layer_device,
-                                                     make_tokens_device)
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py: no CUDA device (there is no CPU path)")
@@ -275,13 +278,67 @@ def run_sfn(args, rank, world, local):
     sfn_build.build()
     L = _capi.lib()
 
-    wl = WORKLOADS[args.workload]
+    K = args.steps if args.steps is not None else default_steps(args.workload)
+    W = max(3, args.warmup if args.warmup is not None else 20)
+    line = measure(args, args.workload, K, W, rank, world, dev, L, main=True)
+    if extra_workloads_wanted(args, world):
+        line_w = {}
+        for name in EXTRA_WORKLOADS:
+            torch.cuda.empty_cache()
+            sub = measure(args, name, default_steps(name, extra=True), W, rank, world, dev, L,
+                          main=False)
+            if sub is not None:
+                line_w[name] = summarize(sub)
+        if line is not None:
+            line["workloads"] = line_w
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+# the other workloads of the metric, measured in the default run beside the
+# headline decode line (each with its own steps, timing, roofline and clocks)
+EXTRA_WORKLOADS = ("batched_decode", "prefill", "long_prefill")
+
+
+def extra_workloads_wanted(args, world):
+    return (args.workloads == "all" and world == 1 and args.workload == "decode"
+            and args.method == "sfn" and args.k is None and args.shard == "tokens"
+            and args.path == "auto")
+
+
+def summarize(line):
+    """The per-workload entry of the headline line."""
+    keys = ("value", "unit", "steps", "warmup", "ms_per_step", "roofline", "step_roofline",
+            "mask_union_channels", "clocks", "gpu_launches", "step_time_spread", "e2e")
+    out = {k: line.get(k) for k in keys}
+    out["workload"] = line["config"]["workload"]
+    out["dtype"] = line["dtype"]
+    out["stages"] = {n: {"us_per_step": v["us_per_step"], "share": v["share"]}
+                     for n, v in line["stages"].items()}
+    return out
+
+
+def measure(args, workload, K, W, rank, world, dev, L, main):
+    """Time K steps of one workload (after W warm-up steps); rank 0 returns
+    its JSON line, the other ranks None."""
+    import numpy as np
+    import torch
+
+    import predictor_gated_channel_b200 as sfn
+    from predictor_gated_channel_b200 import _capi
+    from predictor_gated_channel_b200.inputs import (WORKLOADS, make_layer_device,
+                                                     make_tokens_device)
+    if world > 1:
+        import torch.distributed as dist
+
+    wl = WORKLOADS[workload]
     if args.k is not None:
         wl = wl.with_(k=args.k)
     T = wl.T
-    K = args.steps if args.steps is not None else default_steps(args.workload)
-    W = max(3, args.warmup if args.warmup is not None else 20)
-    S = rotation_layers(args.workload)
+    S = rotation_layers(workload)
     peaks = load_peaks()
 
     shard = args.shard == "banks"
@@ -495,7 +552,7 @@ def run_sfn(args, rank, world, local):
         # timing), under the power cap: the sustained GEMM peak applies
         achieved = work[dom]["flops"] / dom_s / 1e12
         peak, unit = peaks["bf16_tflops_sustained"], "TFLOP/s"
-    traffic = traffic_from_profiles(dom, args.workload)
+    traffic = traffic_from_profiles(dom, workload)
     for n, v in stages.items():
         v["alg_bytes_per_launch"] = work[n]["bytes"]
         v["alg_gbs"] = work[n]["bytes"] / (v["us_per_step"] * 1e-6) / 1e9
@@ -503,7 +560,7 @@ def run_sfn(args, rank, world, local):
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e and not backward and not shard:
-        n_e2e = min(K, 300 if T <= 64 else 10)
+        n_e2e = min(K, 300 if T <= 64 else (10 if main else 3))
         x_host = [xs[i].cpu().pin_memory() for i in range(S)]
         y_host = torch.empty((T, wl.d), dtype=wl.torch_dtype).pin_memory()
         m_host = torch.empty((T, wl.n_banks), dtype=torch.int64).pin_memory()
@@ -541,15 +598,13 @@ def run_sfn(args, rank, world, local):
                "steps": n_e2e}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if main and rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, {k: v.cpu() for k, v in layers[0].items()}, xs[0].cpu(),
                            method=args.method)
 
     if world > 1:
         dist.barrier()
     del g_full, g_rem
-    if world > 1:
-        dist.destroy_process_group()
     if rank != 0:
         return None
 

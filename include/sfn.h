@@ -183,11 +183,16 @@ sfn_status sfn_sparse_ffn_forward_ws(const void *x, const void *A, const void *B
  *   - A shape whose scratch need (sfn_workspace_bytes(..., SFN_DTYPE_BF16))
  *     exceeds SFN_STATIC_SCRATCH_BYTES is rejected with SFN_ERR_WORKSPACE
  *     before anything is enqueued.  For the 4096 x 14336 layer (r 448,
- *     bank 64, k 16) every T up to 265 fits; sfn_workspace_bytes() tells
- *     for any other shape.
+ *     bank 64, k 16) every T up to 81 fits, and T = 129 to 132 (the
+ *     many-token kernels' split sums need more scratch at 82 to 128 tokens
+ *     and from 133); sfn_workspace_bytes() tells for any shape.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  cudaDeviceReset unloads
+ *     the library's module from that device and invalidates the cached
+ *     address (as it does the device error word's, see sfn_device_errors):
+ *     do not call the library on a device after resetting it in the same
+ *     process.
  *   - Every call shares the one array per device.  Calls whose work overlaps
  *     on the GPU (other streams, other host threads) race on it and produce
  *     wrong results: serialise them.  The array keeps the previous call's
@@ -349,9 +354,24 @@ sfn_status sfn_timing_begin(void);
  * two seconds, or a failed index check, sets a bit here and the kernel
  * returns early (its outputs are then invalid).  Bits: 1 = a bounded wait
  * timed out, 2 = an index check failed.  This call synchronises the device,
- * writes the word to *bits and, if `clear`, resets it to 0.
+ * writes the word to *bits and, if `clear`, resets it to 0.  The word's
+ * address is looked up once per device and cached; cudaDeviceReset
+ * invalidates it (and every other per-device cache of the library).
  */
 sfn_status sfn_device_errors(unsigned *bits, int clear);
+
+/*
+ * Self-test of the bounded waits above (diagnostics; no counterpart in the
+ * paper).  Launches one warp on `stream` that waits, through the same
+ * bounded-wait code as every pipeline of this library, on a shared-memory
+ * barrier that nothing ever completes, giving up after `limit_cycles` SM
+ * clock cycles (1 .. 10^9, about half a second at most; else
+ * SFN_ERR_INVALID_VALUE).  The wait then sets bit 1 of the device error word
+ * and the kernel returns; *gave_up (device int, may be NULL) receives 1 if
+ * every lane gave up.  No copy or MMA is in flight, so nothing is left
+ * behind: the device stays usable for later calls.
+ */
+sfn_status sfn_debug_wait_timeout(long long limit_cycles, int *gave_up, sfn_stream_t stream);
 sfn_status sfn_timing_end(double *ms, uint64_t *launches, int n);
 const char *sfn_stage_name(int stage);
 

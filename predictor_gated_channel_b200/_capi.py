@@ -52,6 +52,7 @@ SIGNATURES = {
                                       _vp, _sz, _vp]),
     "sfn_timing_begin": (_ci, []),
     "sfn_device_errors": (_ci, [_vp, _ci]),
+    "sfn_debug_wait_timeout": (_ci, [ctypes.c_longlong, _vp, _vp]),
     "sfn_timing_end": (_ci, [_vp, _vp, _ci]),
     "sfn_stage_name": (ctypes.c_char_p, [_ci]),
 }

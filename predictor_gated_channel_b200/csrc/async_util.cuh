@@ -63,18 +63,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false on timeout
-// (and the timeout is recorded in *err).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err) {
+// Wait for the phase with the given parity to complete, for at most
+// `limit` cycles of SM clock; false on timeout (and the timeout is recorded
+// in *err).
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, unsigned *err,
+                                                long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       report_error(err, kDevErrWaitTimeout);
       return false;
     }
   }
   return true;
+}
+
+// The pipelines' wait: bounded by kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err) {
+  return mbar_wait_limit(bar, parity, err, kWaitLimitCycles);
 }
 
 // 1-D bulk copy global -> shared, completing on `bar` (transaction bytes).

@@ -156,15 +156,32 @@ def test_forward_dense_k64_equals_predictor_gated_dense(full_layer):
     _check_forward(host, x, y, mask, 64, 64, "bf16")
 
 
+def _prefill_rows(T, tile=128):
+    """Rows the oracle checks at a full prefill size.  4096 tokens: every
+    token.  More: one whole 128-token tile in the middle of the grid, the
+    last tile, and one row of every other tile (a different row in each, so
+    every row position inside a tile is covered somewhere)."""
+    if T <= 4096:
+        return np.arange(T)
+    n_tiles = (T + tile - 1) // tile
+    mid = n_tiles // 2
+    rows = set(range(mid * tile, min(T, (mid + 1) * tile)))
+    rows |= set(range((n_tiles - 1) * tile, T))
+    for i in range(n_tiles):
+        rows.add(min(T - 1, i * tile + (i * 37) % tile))
+    return np.array(sorted(rows))
+
+
 @pytest.mark.parametrize("name", ["prefill", "long_prefill"])
-def test_forward_prefill_sampled(name, full_layer):
-    """Full prefill sizes in one call; the oracle checks 40 sampled tokens."""
+def test_forward_prefill(name, full_layer):
+    """Full prefill sizes in one call (the launch configuration the bench
+    times).  At 4096 tokens the oracle checks every token; at 32768 it checks
+    a whole mid-grid tile, the last tile and one row of every other tile."""
     wl = WORKLOADS[name]
     _, host, dev = full_layer
     x = make_tokens(wl)
     y, mask = _run_forward(dev, x.to(DEV), wl.bank, wl.k)
-    rows = np.sort(np.random.default_rng(0).choice(wl.T, 40, replace=False))
-    rows[0], rows[-1] = 0, wl.T - 1
+    rows = _prefill_rows(wl.T)
     _check_forward(host, x, y, mask, wl.bank, wl.k, "bf16", rows=rows)
     assert parity.popcount_ok(parity.to_u64(mask), wl.bank, wl.k)
 
@@ -244,7 +261,7 @@ def test_tensor_path_k_variants(k, full_layer):
     _check_forward(host, x, y, mask, 64, k, "bf16", rows=rows)
 
 
-@pytest.mark.parametrize("k", [1, 4, 16, 20])
+@pytest.mark.parametrize("k", [1, 4, 16, 20, 63])
 def test_tensor_topk_exact_ties(k):
     """One-hot tokens and small-integer A and B make the tensor-core logits
     exact integers; every bank of B holds 16 rows four times each, so exact
@@ -253,24 +270,53 @@ def test_tensor_topk_exact_ties(k):
     16, at 16 and above 16 (the wider-staging variant)."""
     rng = np.random.default_rng(300 + k)
     T, d, d_i, r = 130, 256, 1024, 64
+    x, A, B, W, p = _tie_layer(rng, d, d_i, r, 64, T)
+    _, mask = sfn.sparse_ffn_forward(_bf16_dev(x), _bf16_dev(A), _bf16_dev(B), _bf16_dev(W),
+                                     _bf16_dev(W), _bf16_dev(W), bank=64, k=k, path="tensor")
+    torch.cuda.synchronize()
+    assert np.array_equal(parity.to_u64(mask), oracle.bank_topk(p, 64, k))
+
+
+def _tie_layer(rng, d, d_i, r, bank, T):
+    """One-hot tokens and small-integer A and B, so that the logits are exact
+    integers on either kernel path; inside every bank of B, each of bank/4
+    rows appears four times, so exact ties sit at every threshold."""
     x = np.zeros((T, d), np.float32)
     x[np.arange(T), rng.integers(0, d, T)] = 1.0
     A = rng.integers(-3, 4, (r, d)).astype(np.float32)
     B = rng.integers(-2, 3, (d_i, r)).astype(np.float32)
-    for b in range(d_i // 64):
-        B[b * 64:(b + 1) * 64] = np.tile(B[b * 64:b * 64 + 16], (4, 1))[rng.permutation(64)]
+    q = bank // 4
+    for b in range(d_i // bank):
+        blk = B[b * bank:b * bank + q]
+        B[b * bank:(b + 1) * bank] = np.tile(blk, (4, 1))[rng.permutation(bank)]
     W = (rng.standard_normal((d_i, d)) * 0.05).astype(np.float32)
-
-    def dev_bf16(a):
-        return torch.from_numpy(a).to(torch.bfloat16).to(DEV)
-
-    _, mask = sfn.sparse_ffn_forward(dev_bf16(x), dev_bf16(A), dev_bf16(B), dev_bf16(W),
-                                     dev_bf16(W), dev_bf16(W), bank=64, k=k, path="tensor")
-    torch.cuda.synchronize()
     p = (x.astype(np.int64) @ A.T.astype(np.int64)) @ B.T.astype(np.int64)
     assert np.abs(p).max() < 2 ** 24  # exact in float32
-    want = oracle.bank_topk(p.astype(np.float32), 64, k)
-    assert np.array_equal(parity.to_u64(mask), want)
+    return x, A, B, W, p.astype(np.float32)
+
+
+def _bf16_dev(a):
+    return torch.from_numpy(a).to(torch.bfloat16).to(DEV)
+
+
+@pytest.mark.parametrize("T", [1, 3, 5])
+@pytest.mark.parametrize("bank,k", [(64, 1), (64, 4), (64, 16), (64, 20), (64, 63), (48, 17),
+                                    (32, 5)])
+def test_cuda_core_topk_exact_ties(T, bank, k):
+    """The few-token path ranks each bank inside its logits kernel (a third
+    top-k, beside the standalone one and the tensor-core epilogue).  Fed
+    exact-integer logits with ties everywhere, its mask equals the oracle's
+    bit for bit (ties to the lower channel), for k below, at and above 16,
+    and for banks narrower than 64 (whose order-key rows are padded)."""
+    rng = np.random.default_rng(1000 * bank + 10 * k + T)
+    d, r = 256, 64
+    d_i = (1024 // bank) * bank
+    x, A, B, W, p = _tie_layer(rng, d, d_i, r, bank, T)
+    _, mask = sfn.sparse_ffn_forward(_bf16_dev(x), _bf16_dev(A), _bf16_dev(B), _bf16_dev(W),
+                                     _bf16_dev(W), _bf16_dev(W), bank=bank, k=k,
+                                     path="cuda_core")
+    torch.cuda.synchronize()
+    assert np.array_equal(parity.to_u64(mask), oracle.bank_topk(p, bank, k))
 
 
 def test_paths_agree(full_layer):
