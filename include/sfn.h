@@ -209,19 +209,31 @@ sfn_status sfn_sparse_ffn_forward_static(const void *x, const void *A, const voi
  * Which kernels compute the forward.  The result is the same either way
  * (within rounding; the mask may differ only at exact-threshold ties of the
  * differently rounded logits).
- *   SFN_PATH_CUDA_CORE  gather kernels that read only the kept rows (few
- *                       tokens: every T, any bank <= 64, bf16 or f32);
- *   SFN_PATH_TENSOR     tcgen05 tensor-core GEMMs over 128-token tiles with
- *                       the top-k and the sigma(p) g u mask fused into their
- *                       epilogues (bf16, bank 64, d and d_i multiples of
- *                       256, r a multiple of 64 up to 512);
- *   SFN_PATH_AUTO       the tensor path from T >= 6 when the shape allows
- *                       it, the CUDA-core path otherwise.
+ *   SFN_PATH_CUDA_CORE    gather kernels that read only the kept rows (few
+ *                         tokens: every T, any bank <= 64, bf16 or f32),
+ *                         four launches per call;
+ *   SFN_PATH_TENSOR       tcgen05 tensor-core GEMMs over 128-token tiles with
+ *                         the top-k and the sigma(p) g u mask fused into
+ *                         their epilogues (bf16, bank 64, d and d_i
+ *                         multiples of 256, r a multiple of 64 up to 512);
+ *   SFN_PATH_DECODE_FUSED one token (T = 1, bf16): the same gather kernels'
+ *                         work -- predictor, bank top-k, kept gate/up/down
+ *                         and the final sum -- in one cooperative launch of
+ *                         one CTA per SM (up to 148) with two grid-wide
+ *                         barriers (SFN_ERR_UNSUPPORTED for other T or for a
+ *                         shape outside its shared-memory plan);
+ *   SFN_PATH_AUTO         the fused kernel at T = 1 when the shape allows it,
+ *                         the tensor path from T >= 6 when the shape allows
+ *                         it, the CUDA-core path otherwise.
+ * The fused kernel's barrier state lives in the library and is shared by all
+ * its launches on a device; two of its launches never run at the same time
+ * (each needs every SM), so concurrent calls on other streams are safe.
  */
 typedef enum sfn_path {
   SFN_PATH_AUTO = 0,
   SFN_PATH_CUDA_CORE = 1,
-  SFN_PATH_TENSOR = 2
+  SFN_PATH_TENSOR = 2,
+  SFN_PATH_DECODE_FUSED = 3
 } sfn_path;
 
 /* sfn_sparse_ffn_forward_ws with an explicit path.  SFN_PATH_TENSOR on a
@@ -340,6 +352,7 @@ enum {
   SFN_STAGE_TC_LOGITS_TOPK = 6, /* tensor cores: logits + fused top-k   */
   SFN_STAGE_TC_GATEUP = 7,    /* tensor cores: masked sigma(p) g u      */
   SFN_STAGE_TC_DOWN = 8,      /* tensor cores: y = act W_down           */
+  SFN_STAGE_DECODE_FUSED = 9, /* one token: the whole forward, one launch */
   SFN_STAGE_DENSE4X_GATEUP = 10, /* Dense-4x: silu(g) u + amplitude top-k */
   SFN_STAGE_BWD_TAU = 11,     /* backward: mask and thresholds          */
   SFN_STAGE_BWD_ELEM = 12,    /* backward: surrogate chain rule         */
@@ -354,7 +367,9 @@ sfn_status sfn_timing_begin(void);
  * two seconds, or a failed index check, sets a bit here and the kernel
  * returns early (its outputs are then invalid).  Bits: 1 = a bounded wait
  * timed out, 2 = an index check failed.  This call synchronises the device,
- * writes the word to *bits and, if `clear`, resets it to 0.  The word's
+ * writes the word to *bits and, if `clear`, resets it to 0 (and the fused
+ * decode kernel's grid-barrier state, which a wait that gave up may have left
+ * mid-episode).  The word's
  * address is looked up once per device and cached; cudaDeviceReset
  * invalidates it (and every other per-device cache of the library).
  */

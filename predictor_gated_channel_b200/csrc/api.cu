@@ -246,14 +246,23 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
 // 87 us.
 constexpr int64_t kTcMinTokens = 6;
 bool use_tensor_path(const FwdShape &s, sfn_path path) {
-  if (path == SFN_PATH_CUDA_CORE) return false;
+  if (path == SFN_PATH_CUDA_CORE || path == SFN_PATH_DECODE_FUSED) return false;
   if (!tc_shape_ok(s)) return false;
   return path == SFN_PATH_TENSOR || s.T >= kTcMinTokens;
+}
+
+// One token: the single cooperative kernel, when its shape limits allow
+// (automatic choice), or when asked for.
+bool use_fused_decode(const FwdShape &s, sfn_path path) {
+  if (path != SFN_PATH_AUTO && path != SFN_PATH_DECODE_FUSED) return false;
+  return decode_fused_shape_ok(s, kPlanSms);
 }
 
 size_t workspace_for(const FwdShape &s) {
   size_t need = plan_gather(s).total;
   if (tc_shape_ok(s)) need = std::max(need, plan_tc(s).total);
+  if (decode_fused_shape_ok(s, kPlanSms))
+    need = std::max(need, decode_fused_scratch(s, kPlanSms));
   return need;
 }
 
@@ -264,7 +273,8 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
                         bool y_f32 = false) {
   sfn_status s0 = check_shape(T, d, d_i, r, bank, k);
   if (s0 != SFN_OK) return s0;
-  if (path != SFN_PATH_AUTO && path != SFN_PATH_CUDA_CORE && path != SFN_PATH_TENSOR)
+  if (path != SFN_PATH_AUTO && path != SFN_PATH_CUDA_CORE && path != SFN_PATH_TENSOR &&
+      path != SFN_PATH_DECODE_FUSED)
     return SFN_ERR_INVALID_VALUE;
   if ((s0 = check_limits(d, d_i, r)) != SFN_OK) return s0;
   if ((s0 = check_rows(d, r, bf16)) != SFN_OK) return s0;
@@ -276,9 +286,13 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     return SFN_ERR_MISALIGNED;
   FwdShape s = make_shape(T, d, d_i, r, bank, k, bf16);
   if (path == SFN_PATH_TENSOR && !tc_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
-  const bool tc = use_tensor_path(s, path);
-  if (!tc && !ffn_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
-  const size_t need = tc ? plan_tc(s).total : plan_gather(s).total;
+  if (path == SFN_PATH_DECODE_FUSED && !decode_fused_shape_ok(s, kPlanSms))
+    return SFN_ERR_UNSUPPORTED;
+  const bool fused = use_fused_decode(s, path);
+  const bool tc = !fused && use_tensor_path(s, path);
+  if (!tc && !fused && !ffn_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
+  const size_t need = fused ? decode_fused_scratch(s, kPlanSms)
+                            : (tc ? plan_tc(s).total : plan_gather(s).total);
   if (!own_ws && (ws == nullptr || !aligned(ws, 256) || ws_bytes < need))
     return SFN_ERR_WORKSPACE;
   DeviceInfo dev;
@@ -287,7 +301,11 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     return cuda_status(cudaErrorMemoryAllocation);
   char *w = static_cast<char *>(ws);
   cudaError_t e = cudaSuccess;
-  if (tc) {
+  if (fused) {
+    e = timed(SFN_STAGE_DECODE_FUSED, st, [&] {
+      return launch_decode_fused(s, dev, kPlanSms, x, A, B, Wg, Wu, Wd, y, y_f32, mask, w, st);
+    });
+  } else if (tc) {
     const TcPlan p = plan_tc(s);
     uint16_t *h2 = reinterpret_cast<uint16_t *>(w + p.off_h2);
     float *sig = reinterpret_cast<float *>(w + p.off_sig);
@@ -528,11 +546,17 @@ sfn_status sfn_timing_end(double *ms, uint64_t *launches, int n) {
 sfn_status sfn_device_errors(unsigned *bits, int clear) {
   DeviceInfo dev;
   if (!device_info(&dev)) return SFN_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaErrorUnknown);
   unsigned v = 0;
   if (cudaMemcpy(&v, dev.err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
     return cuda_status(cudaErrorUnknown);
-  if (clear && v != 0 && cudaMemset(dev.err, 0, sizeof v) != cudaSuccess)
-    return cuda_status(cudaErrorUnknown);
+  if (clear && v != 0) {
+    if (cudaMemset(dev.err, 0, sizeof v) != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    // a wait that gave up may have left the fused decode kernel's grid
+    // barrier mid-episode: back to its resting state (the device is idle)
+    if (reset_decode_sync() != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaErrorUnknown);
+  }
   if (bits) *bits = v;
   return SFN_OK;
 }
@@ -780,6 +804,7 @@ const char *sfn_stage_name(int stage) {
     case SFN_STAGE_BWD_ELEM: return "bwd_elem";
     case SFN_STAGE_BWD_GEMM: return "bwd_gemm";
     case SFN_STAGE_BANK_TOPK: return "bank_topk";
+    case SFN_STAGE_DECODE_FUSED: return "decode_fused";
   }
   return "unused";
 }

@@ -316,6 +316,18 @@ cudaError_t launch_bwd_elem(const float *P, const uint64_t *mask, const float *t
                             int bank, float temp, cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float *in, uint16_t *out, int64_t n, cudaStream_t st);
 
+// The one-token forward in one cooperative kernel (decode_fused.cu).  The
+// grid is min(SMs, plan_sms) CTAs; scratch decode_fused_scratch(s, plan_sms).
+bool decode_fused_shape_ok(const FwdShape &s, int G);
+size_t decode_fused_scratch(const FwdShape &s, int G);
+cudaError_t launch_decode_fused(const FwdShape &s, const DeviceInfo &dev, int plan_sms,
+                                const void *x, const void *A, const void *B, const void *Wg,
+                                const void *Wu, const void *Wd, void *y, bool y_f32,
+                                uint64_t *mask, void *scratch, cudaStream_t st);
+// Back to the resting state of the fused kernel's grid barrier (after a
+// timeout left it inconsistent); the device must be idle.
+cudaError_t reset_decode_sync();
+
 // Scratch carve-up of the tensor-core path.
 struct TcPlan {
   int ksplit;  // K ranges of the down GEMM (fp32 partials reduced after)
