@@ -223,11 +223,14 @@ def test_outputs_do_not_spill(full_layer):
 
 
 def test_launch_counter_counts_kernels(full_layer):
+    """One token: the single fused kernel; two tokens: the four few-token
+    kernels."""
     wl, host, dev = full_layer
-    x = make_tokens(wl, T=1).to(DEV)
-    c0 = sfn.kernel_launch_count()
-    _run_forward(dev, x, 64, 16)
-    assert sfn.kernel_launch_count() - c0 >= 3
+    for T, n in ((1, 1), (2, 4)):
+        x = make_tokens(wl, T=T).to(DEV)
+        c0 = sfn.kernel_launch_count()
+        _run_forward(dev, x, 64, 16)
+        assert sfn.kernel_launch_count() - c0 == n, T
 
 
 def test_zero_tokens(full_layer):
