@@ -63,7 +63,7 @@ def parse_args(argv=None):
     ap.add_argument("--temperature", type=float, default=1.0,
                     help="surrogate temperature of --method backward")
     ap.add_argument("--path", default="auto",
-                    choices=["auto", "cuda_core", "tensor", "decode_fused"],
+                    choices=["auto", "cuda_core", "tensor"],
                     help="kernels to use (the library picks by token count when auto)")
     ap.add_argument("--workloads", default="all", choices=["all", "one"],
                     help="all (default): with the default decode workload, also measure the "
@@ -177,7 +177,7 @@ def _num(s):
 # stage name -> the source files that define its kernel
 KERNEL_SOURCES = {
     "pred_h": ["predict_topk.cu"], "logits_topk": ["predict_topk.cu"],
-    "ffn": ["gather_ffn.cu"], "reduce": ["gather_ffn.cu"], "decode_fused": ["decode_fused.cu"],
+    "ffn": ["gather_ffn.cu"], "reduce": ["gather_ffn.cu"],
     "tc_h": ["tc_path.cu", "tc_util.cuh"], "tc_logits_topk": ["tc_path.cu", "tc_util.cuh"],
     "tc_gateup": ["tc_path.cu", "tc_util.cuh"], "tc_down": ["tc_path.cu", "tc_util.cuh"],
 }
@@ -228,10 +228,6 @@ def stage_work(wl, T, union_channels):
            "flops": 6 * T * d_s * d}
     return {
         "pred_h": pred_h, "logits_topk": logits, "ffn": ffn,
-        # one token in one launch: predictor weights, kept rows, x and y
-        "decode_fused": {"bytes": r * d * e + d_i * r * e + 3 * union_channels * d * e
-                                  + 2 * T * d * e,
-                         "flops": 2 * T * (d * r + r * d_i + 3 * d_s * d)},
         "reduce": {"bytes": T * d * e, "flops": 0},
         "tc_h": pred_h, "tc_logits_topk": logits,
         "tc_gateup": {"bytes": 2 * union_channels * d * e + T * d * e + T * d_i * e,
@@ -382,7 +378,7 @@ def measure(args, workload, K, W, rank, world, dev, L, main):
     else:
         ws_bytes = sfn.workspace_bytes(T, wl.d, wl.d_i, wl.r, wl.bank, wl.k, wl.torch_dtype)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    path_id = {"auto": 0, "cuda_core": 1, "tensor": 2, "decode_fused": 3}[args.path]
+    path_id = {"auto": 0, "cuda_core": 1, "tensor": 2}[args.path]
     stream = torch.cuda.Stream(device=dev)
 
     def call(i, st_ptr):

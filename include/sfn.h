@@ -50,12 +50,10 @@
  * without synchronising; results are ready when the stream is.  No call
  * copies between host and device.  The only allocations are the
  * stream-ordered scratch of sfn_sparse_ffn_forward and sfn_predict
- * (cudaMallocAsync / cudaFreeAsync on `stream`) and, on the first backward
- * call on a device, the cuBLAS handle it creates; the other entry points
+ * (cudaMallocAsync / cudaFreeAsync on `stream`); the other entry points
  * take caller scratch.  Calls on different streams may run concurrently if
  * their outputs and scratch do not overlap.  Results are deterministic: a
- * fixed reduction order and no floating-point atomics (the backward's
- * cuBLAS GEMMs are deterministic for a given GPU), so a rerun is
+ * fixed reduction order and no floating-point atomics, so a rerun is
  * bit-identical.
  *
  * Errors: every argument is checked on the host before anything is
@@ -108,9 +106,8 @@ const char *sfn_status_string(sfn_status s);
 /* ABI version of this header (incremented on any signature change). */
 int sfn_abi_version(void);
 
-/* The message behind the last SFN_ERR_CUDA (the CUDA runtime's) or the last
- * SFN_ERR_UNSUPPORTED of the backward (why cuBLAS could not be loaded)
- * returned on this host thread (static string; "no error" if none). */
+/* The message behind the last SFN_ERR_CUDA (the CUDA runtime's) returned on
+ * this host thread (static string; "no error" if none). */
 const char *sfn_last_error_string(void);
 
 /* Number of kernels this library has launched in this process (all
@@ -209,31 +206,28 @@ sfn_status sfn_sparse_ffn_forward_static(const void *x, const void *A, const voi
  * Which kernels compute the forward.  The result is the same either way
  * (within rounding; the mask may differ only at exact-threshold ties of the
  * differently rounded logits).
- *   SFN_PATH_CUDA_CORE    gather kernels that read only the kept rows (few
- *                         tokens: every T, any bank <= 64, bf16 or f32),
- *                         four launches per call;
- *   SFN_PATH_TENSOR       tcgen05 tensor-core GEMMs over 128-token tiles with
- *                         the top-k and the sigma(p) g u mask fused into
- *                         their epilogues (bf16, bank 64, d and d_i
- *                         multiples of 256, r a multiple of 64 up to 512);
- *   SFN_PATH_DECODE_FUSED one token (T = 1, bf16): the same gather kernels'
- *                         work -- predictor, bank top-k, kept gate/up/down
- *                         and the final sum -- in one cooperative launch of
- *                         one CTA per SM (up to 148) with two grid-wide
- *                         barriers (SFN_ERR_UNSUPPORTED for other T or for a
- *                         shape outside its shared-memory plan);
- *   SFN_PATH_AUTO         the fused kernel at T = 1 when the shape allows it,
- *                         the tensor path from T >= 6 when the shape allows
- *                         it, the CUDA-core path otherwise.
- * The fused kernel's barrier state lives in the library and is shared by all
- * its launches on a device; two of its launches never run at the same time
- * (each needs every SM), so concurrent calls on other streams are safe.
+ *   SFN_PATH_CUDA_CORE  gather kernels that read only the kept rows (few
+ *                       tokens: every T, any bank <= 64, bf16 or f32); when
+ *                       all of the call's gate/up/down CTAs fit the device at
+ *                       once (T <= 5 on a B200), the final sum of their
+ *                       partial rows runs in the same cooperative launch
+ *                       after a grid-wide barrier, else in a kernel of its
+ *                       own;
+ *   SFN_PATH_TENSOR     tcgen05 tensor-core GEMMs over 128-token tiles with
+ *                       the top-k and the sigma(p) g u mask fused into their
+ *                       epilogues (bf16, bank 64, d and d_i multiples of
+ *                       256, r a multiple of 64 up to 512);
+ *   SFN_PATH_AUTO       the tensor path from T >= 6 when the shape allows
+ *                       it, the CUDA-core path otherwise.
+ * The cooperative launch's barrier state lives in the library and is shared
+ * by its launches on a device; two of them never run at the same time (each
+ * takes one CTA on every SM it uses, and cooperative grids are placed only
+ * when all their CTAs fit), so concurrent calls on other streams stay safe.
  */
 typedef enum sfn_path {
   SFN_PATH_AUTO = 0,
   SFN_PATH_CUDA_CORE = 1,
-  SFN_PATH_TENSOR = 2,
-  SFN_PATH_DECODE_FUSED = 3
+  SFN_PATH_TENSOR = 2
 } sfn_path;
 
 /* sfn_sparse_ffn_forward_ws with an explicit path.  SFN_PATH_TENSOR on a
@@ -305,10 +299,10 @@ sfn_status sfn_dense4x_forward(const void *x, const void *Wg, const void *Wu, co
  * bf16 inputs (x, A, B, Wg, Wu, Wd, dy); logits are recomputed with the
  * forward's own kernels (the same mask as the forward for the same T), the
  * elementwise chain rule runs in this library's kernels, and the dense
- * contractions use cuBLAS (bf16 operands, float32 accumulation), loaded at
- * run time: SFN_ERR_UNSUPPORTED if libcublas.so.12 cannot be loaded.
- * temperature must be finite and > 0 (else SFN_ERR_INVALID_VALUE); d_i must
- * be a multiple of 4.  Scratch: at least sfn_backward_workspace_bytes()
+ * contractions run on its tcgen05 tensor-core GEMM (bf16 operands, float32
+ * accumulation and output).  temperature must be finite and > 0 (else
+ * SFN_ERR_INVALID_VALUE); d, d_i and r must be multiples of 64 (else
+ * SFN_ERR_UNSUPPORTED).  Scratch: at least sfn_backward_workspace_bytes()
  * bytes, 256-byte aligned (1.4 GB for 4096 tokens of the 4096 x 14336
  * layer).  Other errors as sfn_sparse_ffn_forward_ws.
  */
@@ -345,18 +339,19 @@ sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const f
 enum {
   SFN_STAGE_PRED_H = 0,       /* h = A x                                */
   SFN_STAGE_LOGITS_TOPK = 1,  /* p = B h, bank top-k, sigma(p) of kept  */
-  SFN_STAGE_FFN = 2,          /* kept gate/up/down rows -> partial y    */
+  SFN_STAGE_FFN = 2,          /* kept gate/up/down rows -> partial y
+                                 (and y itself, when summed in the same
+                                 cooperative launch)                    */
   SFN_STAGE_REDUCE = 3,       /* partial rows -> y (few tokens)         */
   SFN_STAGE_BANK_TOPK = 4,    /* standalone top-k on given logits       */
   SFN_STAGE_TC_H = 5,         /* tensor cores: h = A x, split hi/lo     */
   SFN_STAGE_TC_LOGITS_TOPK = 6, /* tensor cores: logits + fused top-k   */
   SFN_STAGE_TC_GATEUP = 7,    /* tensor cores: masked sigma(p) g u      */
   SFN_STAGE_TC_DOWN = 8,      /* tensor cores: y = act W_down           */
-  SFN_STAGE_DECODE_FUSED = 9, /* one token: the whole forward, one launch */
   SFN_STAGE_DENSE4X_GATEUP = 10, /* Dense-4x: silu(g) u + amplitude top-k */
   SFN_STAGE_BWD_TAU = 11,     /* backward: mask and thresholds          */
   SFN_STAGE_BWD_ELEM = 12,    /* backward: surrogate chain rule         */
-  SFN_STAGE_BWD_GEMM = 13,    /* backward: cuBLAS contractions          */
+  SFN_STAGE_BWD_GEMM = 13,    /* backward: tensor-core contractions     */
   SFN_STAGE_COUNT = 16        /* room for the stage ids of this library */
 };
 sfn_status sfn_timing_begin(void);
@@ -367,9 +362,9 @@ sfn_status sfn_timing_begin(void);
  * two seconds, or a failed index check, sets a bit here and the kernel
  * returns early (its outputs are then invalid).  Bits: 1 = a bounded wait
  * timed out, 2 = an index check failed.  This call synchronises the device,
- * writes the word to *bits and, if `clear`, resets it to 0 (and the fused
- * decode kernel's grid-barrier state, which a wait that gave up may have left
- * mid-episode).  The word's
+ * writes the word to *bits and, if `clear`, resets it to 0 (and the
+ * grid-barrier state of the cooperative gate/up/down kernel, which a wait
+ * that gave up may have left mid-episode).  The word's
  * address is looked up once per device and cached; cudaDeviceReset
  * invalidates it (and every other per-device cache of the library).
  */

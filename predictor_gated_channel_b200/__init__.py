@@ -95,7 +95,7 @@ def bank_topk(logits, bank: int = 64, k: int = 16, out=None, stream=None):
 
 
 PATHS = {"auto": _capi.SFN_PATH_AUTO, "cuda_core": _capi.SFN_PATH_CUDA_CORE,
-         "tensor": _capi.SFN_PATH_TENSOR, "decode_fused": _capi.SFN_PATH_DECODE_FUSED}
+         "tensor": _capi.SFN_PATH_TENSOR}
 
 
 def sparse_ffn_forward(x, A, B, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None, mask=None,
@@ -106,7 +106,7 @@ def sparse_ffn_forward(x, A, B, Wg, Wu, Wd, bank: int = 64, k: int = 16, y=None,
     Returns (y [T, d] in x's dtype, mask int64 [T, d_i/bank] or None).  With
     ``workspace`` (a uint8 CUDA tensor of at least ``workspace_bytes(...)``)
     the call uses it as scratch instead of allocating stream-ordered memory.
-    ``path`` ("auto", "cuda_core", "tensor" or "decode_fused") picks the kernels; a bf16
+    ``path`` ("auto", "cuda_core" or "tensor") picks the kernels; a bf16
     call with an explicit path always uses caller scratch (allocated here
     when ``workspace`` is None).
     """

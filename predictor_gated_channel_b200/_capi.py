@@ -20,7 +20,6 @@ SFN_ERR_CUDA = 5
 SFN_PATH_AUTO = 0
 SFN_PATH_CUDA_CORE = 1
 SFN_PATH_TENSOR = 2
-SFN_PATH_DECODE_FUSED = 3
 
 SFN_DTYPE_BF16 = 0
 SFN_DTYPE_F32 = 1

@@ -246,23 +246,14 @@ sfn_status predict_impl(const void *x, const void *A, const void *B, float *logi
 // 87 us.
 constexpr int64_t kTcMinTokens = 6;
 bool use_tensor_path(const FwdShape &s, sfn_path path) {
-  if (path == SFN_PATH_CUDA_CORE || path == SFN_PATH_DECODE_FUSED) return false;
+  if (path == SFN_PATH_CUDA_CORE) return false;
   if (!tc_shape_ok(s)) return false;
   return path == SFN_PATH_TENSOR || s.T >= kTcMinTokens;
-}
-
-// One token: the single cooperative kernel, when its shape limits allow
-// (automatic choice), or when asked for.
-bool use_fused_decode(const FwdShape &s, sfn_path path) {
-  if (path != SFN_PATH_AUTO && path != SFN_PATH_DECODE_FUSED) return false;
-  return decode_fused_shape_ok(s, kPlanSms);
 }
 
 size_t workspace_for(const FwdShape &s) {
   size_t need = plan_gather(s).total;
   if (tc_shape_ok(s)) need = std::max(need, plan_tc(s).total);
-  if (decode_fused_shape_ok(s, kPlanSms))
-    need = std::max(need, decode_fused_scratch(s, kPlanSms));
   return need;
 }
 
@@ -273,8 +264,7 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
                         bool y_f32 = false) {
   sfn_status s0 = check_shape(T, d, d_i, r, bank, k);
   if (s0 != SFN_OK) return s0;
-  if (path != SFN_PATH_AUTO && path != SFN_PATH_CUDA_CORE && path != SFN_PATH_TENSOR &&
-      path != SFN_PATH_DECODE_FUSED)
+  if (path != SFN_PATH_AUTO && path != SFN_PATH_CUDA_CORE && path != SFN_PATH_TENSOR)
     return SFN_ERR_INVALID_VALUE;
   if ((s0 = check_limits(d, d_i, r)) != SFN_OK) return s0;
   if ((s0 = check_rows(d, r, bf16)) != SFN_OK) return s0;
@@ -286,13 +276,9 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     return SFN_ERR_MISALIGNED;
   FwdShape s = make_shape(T, d, d_i, r, bank, k, bf16);
   if (path == SFN_PATH_TENSOR && !tc_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
-  if (path == SFN_PATH_DECODE_FUSED && !decode_fused_shape_ok(s, kPlanSms))
-    return SFN_ERR_UNSUPPORTED;
-  const bool fused = use_fused_decode(s, path);
-  const bool tc = !fused && use_tensor_path(s, path);
-  if (!tc && !fused && !ffn_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
-  const size_t need = fused ? decode_fused_scratch(s, kPlanSms)
-                            : (tc ? plan_tc(s).total : plan_gather(s).total);
+  const bool tc = use_tensor_path(s, path);
+  if (!tc && !ffn_shape_ok(s)) return SFN_ERR_UNSUPPORTED;
+  const size_t need = tc ? plan_tc(s).total : plan_gather(s).total;
   if (!own_ws && (ws == nullptr || !aligned(ws, 256) || ws_bytes < need))
     return SFN_ERR_WORKSPACE;
   DeviceInfo dev;
@@ -301,11 +287,7 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     return cuda_status(cudaErrorMemoryAllocation);
   char *w = static_cast<char *>(ws);
   cudaError_t e = cudaSuccess;
-  if (fused) {
-    e = timed(SFN_STAGE_DECODE_FUSED, st, [&] {
-      return launch_decode_fused(s, dev, kPlanSms, x, A, B, Wg, Wu, Wd, y, y_f32, mask, w, st);
-    });
-  } else if (tc) {
+  if (tc) {
     const TcPlan p = plan_tc(s);
     uint16_t *h2 = reinterpret_cast<uint16_t *>(w + p.off_h2);
     float *sig = reinterpret_cast<float *>(w + p.off_sig);
@@ -358,16 +340,24 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
       e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
         return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, dev.err, st);
       });
-    if (e == cudaSuccess)
-      e = timed(SFN_STAGE_FFN, st, [&] {
-        return launch_ffn(s, p.cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, dev.err, st);
-      });
-    if (e == cudaSuccess)
-      e = timed(SFN_STAGE_REDUCE, st,
-                [&] {
-                  return launch_reduce_partials(s, p.cpt, partial, y, st,
-                                                y_f32 ? ReduceOut::kYF32 : ReduceOut::kY);
-                });
+    if (ffn_sum_ok(s, p.cpt, dev)) {
+      // gate/up/down and the sum of the partial rows in one cooperative launch
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_FFN, st, [&] {
+          return launch_ffn_sum(s, p.cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, y, y_f32,
+                                dev.err, st);
+        });
+    } else {
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_FFN, st, [&] {
+          return launch_ffn(s, p.cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, dev.err, st);
+        });
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_REDUCE, st, [&] {
+          return launch_reduce_partials(s, p.cpt, partial, y, st,
+                                        y_f32 ? ReduceOut::kYF32 : ReduceOut::kY);
+        });
+    }
   }
   if (own_ws) {
     cudaError_t ef = cudaFreeAsync(ws, st);
@@ -552,9 +542,10 @@ sfn_status sfn_device_errors(unsigned *bits, int clear) {
     return cuda_status(cudaErrorUnknown);
   if (clear && v != 0) {
     if (cudaMemset(dev.err, 0, sizeof v) != cudaSuccess) return cuda_status(cudaErrorUnknown);
-    // a wait that gave up may have left the fused decode kernel's grid
-    // barrier mid-episode: back to its resting state (the device is idle)
-    if (reset_decode_sync() != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    // a wait that gave up may have left the cooperative gate/up/down
+    // kernel's grid barrier mid-episode: back to its resting state (the
+    // device is idle)
+    if (reset_grid_sync() != cudaSuccess) return cuda_status(cudaErrorUnknown);
     if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaErrorUnknown);
   }
   if (bits) *bits = v;
@@ -654,7 +645,9 @@ sfn_status check_backward(int64_t T, int d, int d_i, int r, int bank, int k, flo
   if (!(temp > 0.f) || !std::isfinite(temp)) return SFN_ERR_INVALID_VALUE;
   if ((s0 = check_limits(d, d_i, r)) != SFN_OK) return s0;
   if ((s0 = check_rows(d, r, true)) != SFN_OK) return s0;
-  if (d_i % 4 != 0 || T > 0x7fffffffLL) return SFN_ERR_UNSUPPORTED;
+  // the tensor-core contractions take N in multiples of 64 (N is d, d_i or r)
+  if (d % 64 != 0 || d_i % 64 != 0 || r % 64 != 0 || T > 0x7fffffffLL)
+    return SFN_ERR_UNSUPPORTED;
   return SFN_OK;
 }
 }  // namespace
@@ -672,11 +665,6 @@ sfn_status sfn_sparse_ffn_backward(const void *x, const void *A, const void *B, 
                                    void *ws, size_t ws_bytes, sfn_stream_t stream) {
   sfn_status s0 = check_backward(T, d, d_i, r, bank, k, temperature);
   if (s0 != SFN_OK) return s0;
-  const char *why = nullptr;
-  if (!blas_available(&why)) {
-    t_last_error = why;
-    return SFN_ERR_UNSUPPORTED;
-  }
   if (T == 0) return SFN_OK;
   if (!x || !A || !B || !Wg || !Wu || !Wd || !dy) return SFN_ERR_INVALID_VALUE;
   for (const void *q : {x, A, B, Wg, Wu, Wd, dy, (const void *)dx, (const void *)dA,
@@ -742,17 +730,20 @@ sfn_status sfn_sparse_ffn_backward(const void *x, const void *A, const void *B, 
   if (e == cudaSuccess && !p.tc)
     e = timed(SFN_STAGE_BWD_TAU, st,
               [&] { return launch_bank_tau(P, m, tau, T, d_i, bank, k, st); });
-  BlasLock blas;
-  // 3. g, u (every channel) and da = Wd dy, float32 [T][d_i]
-  auto gemm = [&](bool ta, bool tb, int mm, int nn, int kk, const void *Am, int lda,
-                  const void *Bm, int ldb, float *C, int ldc, float beta) {
-    return blas_gemm_bf16(dev.device, st, ta, tb, mm, nn, kk, Am, lda, Bm, ldb, C, ldc, beta);
+  // The contractions run on this library's tcgen05 GEMM (bf16 operands,
+  // float32 accumulate and output).  gemm(M, N, K, A, lda, a_mn, B, ldb, b_mn,
+  // C, ldc, acc): C[M][N] (+)= A B with A [M][K] or [K][M] (a_mn), B [N][K]
+  // or [K][N] (b_mn).
+  auto gemm = [&](int mm, int nn, int kk, const void *Am, int lda, bool a_mn, const void *Bm,
+                  int ldb, bool b_mn, float *C, int ldc, bool acc) {
+    return launch_tc_gemm_f32(dev, mm, nn, kk, Am, lda, a_mn, Bm, ldb, b_mn, C, ldc, acc, st);
   };
+  // 3. g = Wg x, u = Wu x (every channel) and da = Wd dy, float32 [T][d_i]
   if (e == cudaSuccess)
     e = timed(SFN_STAGE_BWD_GEMM, st, [&] {
-      cudaError_t r1 = gemm(true, false, d_i, Ti, d, Wg, d, x, d, G, d_i, 0.f);
-      if (r1 == cudaSuccess) r1 = gemm(true, false, d_i, Ti, d, Wu, d, x, d, U, d_i, 0.f);
-      if (r1 == cudaSuccess) r1 = gemm(true, false, d_i, Ti, d, Wd, d, dy, d, DA, d_i, 0.f);
+      cudaError_t r1 = gemm(Ti, d_i, d, x, d, false, Wg, d, false, G, d_i, false);
+      if (r1 == cudaSuccess) r1 = gemm(Ti, d_i, d, x, d, false, Wu, d, false, U, d_i, false);
+      if (r1 == cudaSuccess) r1 = gemm(Ti, d_i, d, dy, d, false, Wd, d, false, DA, d_i, false);
       return r1;
     });
   // 4. the chain rule with the surrogate
@@ -761,28 +752,35 @@ sfn_status sfn_sparse_ffn_backward(const void *x, const void *A, const void *B, 
       return launch_bwd_elem(P, m, tau, G, U, DA, a, dg, du, dp, T, d_i, bank, temperature,
                              st);
     });
-  // 5. contractions back to the inputs
+  // 5. contractions back to the inputs; the weight gradients contract over
+  // the tokens (K = T), with both operands stored token-major
   const bool need_dh = dA != nullptr || dx != nullptr;
   if (e == cudaSuccess)
     e = timed(SFN_STAGE_BWD_GEMM, st, [&] {
       cudaError_t r1 = cudaSuccess;
-      if (dWd) r1 = gemm(false, true, d, d_i, Ti, dy, d, a, d_i, dWd, d, 0.f);
-      if (r1 == cudaSuccess && dWg) r1 = gemm(false, true, d, d_i, Ti, x, d, dg, d_i, dWg, d, 0.f);
-      if (r1 == cudaSuccess && dWu) r1 = gemm(false, true, d, d_i, Ti, x, d, du, d_i, dWu, d, 0.f);
-      if (r1 == cudaSuccess && dB) r1 = gemm(false, true, r, d_i, Ti, hb, ldh, dp, d_i, dB, r, 0.f);
+      // dWd[j][n] = sum_t a[t][j] dy[t][n]
+      if (dWd) r1 = gemm(d_i, d, Ti, a, d_i, true, dy, d, true, dWd, d, false);
+      // dWg[j][n] = sum_t dg[t][j] x[t][n]; dWu likewise with du
+      if (r1 == cudaSuccess && dWg) r1 = gemm(d_i, d, Ti, dg, d_i, true, x, d, true, dWg, d, false);
+      if (r1 == cudaSuccess && dWu) r1 = gemm(d_i, d, Ti, du, d_i, true, x, d, true, dWu, d, false);
+      // dB[j][m] = sum_t dp[t][j] h[t][m]
+      if (r1 == cudaSuccess && dB) r1 = gemm(d_i, r, Ti, dp, d_i, true, hb, ldh, true, dB, r, false);
+      // dh[t][m] = sum_j dp[t][j] B[j][m]
       if (r1 == cudaSuccess && need_dh)
-        r1 = gemm(false, false, r, Ti, d_i, B, r, dp, d_i, dH, r, 0.f);
+        r1 = gemm(Ti, r, d_i, dp, d_i, false, B, r, true, dH, r, false);
       return r1;
     });
   if (e == cudaSuccess && need_dh) e = launch_f32_to_bf16(dH, dHb, T * r, st);
   if (e == cudaSuccess && need_dh)
     e = timed(SFN_STAGE_BWD_GEMM, st, [&] {
       cudaError_t r1 = cudaSuccess;
-      if (dA) r1 = gemm(false, true, d, r, Ti, x, d, dHb, r, dA, d, 0.f);
+      // dA[m][n] = sum_t dh[t][m] x[t][n]
+      if (dA) r1 = gemm(r, d, Ti, dHb, r, true, x, d, true, dA, d, false);
+      // dx = dg Wg + du Wu + dh A, accumulated in float32
       if (r1 == cudaSuccess && dx) {
-        r1 = gemm(false, false, d, Ti, d_i, Wg, d, dg, d_i, dx, d, 0.f);
-        if (r1 == cudaSuccess) r1 = gemm(false, false, d, Ti, d_i, Wu, d, du, d_i, dx, d, 1.f);
-        if (r1 == cudaSuccess) r1 = gemm(false, false, d, Ti, r, A, d, dHb, r, dx, d, 1.f);
+        r1 = gemm(Ti, d, d_i, dg, d_i, false, Wg, d, true, dx, d, false);
+        if (r1 == cudaSuccess) r1 = gemm(Ti, d, d_i, du, d_i, false, Wu, d, true, dx, d, true);
+        if (r1 == cudaSuccess) r1 = gemm(Ti, d, r, dHb, r, false, A, d, true, dx, d, true);
       }
       return r1;
     });
@@ -804,7 +802,6 @@ const char *sfn_stage_name(int stage) {
     case SFN_STAGE_BWD_ELEM: return "bwd_elem";
     case SFN_STAGE_BWD_GEMM: return "bwd_gemm";
     case SFN_STAGE_BANK_TOPK: return "bank_topk";
-    case SFN_STAGE_DECODE_FUSED: return "decode_fused";
   }
   return "unused";
 }

@@ -21,15 +21,9 @@
 //   k_f32_to_bf16 float32 -> bf16 rows (h and dh as GEMM operands)
 //
 // The dense contractions around them (g, u, da; the weight gradients; dh,
-// dx) are plain GEMMs and go to cuBLAS (bf16 operands, float32 accumulate
-// and output), loaded at run time so that the library itself does not
-// depend on it.
-#include <dlfcn.h>
-
+// dx) run on the library's tcgen05 GEMM (tc_path.cu, launch_tc_gemm_f32:
+// bf16 operands, float32 accumulation and output).
 #include <cmath>
-#include <mutex>
-
-#include <cublas_v2.h>
 
 #include "sfn_internal.cuh"
 
@@ -162,73 +156,7 @@ __global__ void __launch_bounds__(kElemThreads) k_f32_to_bf16(const float *__res
   if (i < n) out[i] = f32_to_bf16_bits(in[i]);
 }
 
-// ------------------------------------------------------------------ cuBLAS
-// Resolved once from libcublas.so.12; calls are serialised (one handle per
-// device, not shared between threads at the same time).
-using CreateFn = cublasStatus_t (*)(cublasHandle_t *);
-using SetStreamFn = cublasStatus_t (*)(cublasHandle_t, cudaStream_t);
-using GemmExFn = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int,
-                                    int, int, const void *, const void *, cudaDataType, int,
-                                    const void *, cudaDataType, int, const void *, void *,
-                                    cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t);
-struct Cublas {
-  bool ok = false;
-  const char *why = "cuBLAS not loaded";
-  CreateFn create = nullptr;
-  SetStreamFn set_stream = nullptr;
-  GemmExFn gemm = nullptr;
-  cublasHandle_t handle[64] = {};
-};
-Cublas g_blas;
-std::once_flag g_blas_once;
-std::mutex g_blas_mu;
-
-void load_cublas() {
-  void *h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
-  if (h == nullptr) {
-    g_blas.why = "libcublas.so.12 could not be loaded";
-    return;
-  }
-  g_blas.create = reinterpret_cast<CreateFn>(dlsym(h, "cublasCreate_v2"));
-  g_blas.set_stream = reinterpret_cast<SetStreamFn>(dlsym(h, "cublasSetStream_v2"));
-  g_blas.gemm = reinterpret_cast<GemmExFn>(dlsym(h, "cublasGemmEx"));
-  if (!g_blas.create || !g_blas.set_stream || !g_blas.gemm) {
-    g_blas.why = "libcublas.so.12 lacks a needed entry point";
-    return;
-  }
-  g_blas.ok = true;
-  g_blas.why = "ok";
-}
-
 }  // namespace
-
-bool blas_available(const char **why) {
-  std::call_once(g_blas_once, load_cublas);
-  if (why) *why = g_blas.why;
-  return g_blas.ok;
-}
-
-BlasLock::BlasLock() : lock_(g_blas_mu) {}
-BlasLock::~BlasLock() = default;
-
-cudaError_t blas_gemm_bf16(int device, cudaStream_t st, bool ta, bool tb, int m, int n, int k,
-                           const void *A, int lda, const void *B, int ldb, float *C, int ldc,
-                           float beta) {
-  if (!blas_available(nullptr) || device < 0 || device >= 64) return cudaErrorNotSupported;
-  if (m == 0 || n == 0) return cudaSuccess;
-  cublasHandle_t &hd = g_blas.handle[device];
-  if (hd == nullptr && g_blas.create(&hd) != CUBLAS_STATUS_SUCCESS) {
-    hd = nullptr;
-    return cudaErrorNotSupported;
-  }
-  if (g_blas.set_stream(hd, st) != CUBLAS_STATUS_SUCCESS) return cudaErrorUnknown;
-  const float alpha = 1.f;
-  const cublasStatus_t s =
-      g_blas.gemm(hd, ta ? CUBLAS_OP_T : CUBLAS_OP_N, tb ? CUBLAS_OP_T : CUBLAS_OP_N, m, n, k,
-                  &alpha, A, CUDA_R_16BF, lda, B, CUDA_R_16BF, ldb, &beta, C, CUDA_R_32F, ldc,
-                  CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-  return s == CUBLAS_STATUS_SUCCESS ? cudaSuccess : cudaErrorUnknown;
-}
 
 cudaError_t launch_bank_tau(const float *logits, uint64_t *mask, float *tau, int64_t T, int d_i,
                             int bank, int k, cudaStream_t st) {

@@ -290,24 +290,21 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
 // kYF32: y as float32 whatever the input type (partial outputs of a bank
 // shard, summed across devices before rounding).
 enum class ReduceOut { kY, kYF32, kSplitH };
+// The few-token gate/up/down with the final sum in the same cooperative
+// launch (k_ffn_sum, T * cpt CTAs, one per SM): y (bf16 or float32 per the
+// call) instead of partial rows for a separate sum.  ffn_sum_ok tells whether
+// the grid fits the device; reset_grid_sync returns its grid barrier to the
+// resting state after a wait gave up (the device must be idle).
+bool ffn_sum_ok(const FwdShape &s, int cpt, const DeviceInfo &dev);
+cudaError_t launch_ffn_sum(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
+                           const float *sel_sig, const void *Wg, const void *Wu,
+                           const void *Wd, float *partial, void *y, bool y_f32, unsigned *err,
+                           cudaStream_t st);
+cudaError_t reset_grid_sync();
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
                                    cudaStream_t st, ReduceOut kind = ReduceOut::kY);
 
 // ---------------------------------------------------------------- backward
-// cuBLAS, loaded at run time for the backward's plain GEMMs (bf16 operands,
-// float32 accumulate and output, column-major as cuBLAS sees it).  Hold a
-// BlasLock while enqueuing a sequence of blas_gemm_bf16 calls.
-bool blas_available(const char **why);
-class BlasLock {
- public:
-  BlasLock();
-  ~BlasLock();
- private:
-  std::lock_guard<std::mutex> lock_;
-};
-cudaError_t blas_gemm_bf16(int device, cudaStream_t st, bool ta, bool tb, int m, int n, int k,
-                           const void *A, int lda, const void *B, int ldb, float *C, int ldc,
-                           float beta);
 cudaError_t launch_bank_tau(const float *logits, uint64_t *mask, float *tau, int64_t T, int d_i,
                             int bank, int k, cudaStream_t st);
 cudaError_t launch_bwd_elem(const float *P, const uint64_t *mask, const float *tau,
@@ -315,18 +312,6 @@ cudaError_t launch_bwd_elem(const float *P, const uint64_t *mask, const float *t
                             uint16_t *dg, uint16_t *du, uint16_t *dp, int64_t T, int d_i,
                             int bank, float temp, cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float *in, uint16_t *out, int64_t n, cudaStream_t st);
-
-// The one-token forward in one cooperative kernel (decode_fused.cu).  The
-// grid is min(SMs, plan_sms) CTAs; scratch decode_fused_scratch(s, plan_sms).
-bool decode_fused_shape_ok(const FwdShape &s, int G);
-size_t decode_fused_scratch(const FwdShape &s, int G);
-cudaError_t launch_decode_fused(const FwdShape &s, const DeviceInfo &dev, int plan_sms,
-                                const void *x, const void *A, const void *B, const void *Wg,
-                                const void *Wu, const void *Wd, void *y, bool y_f32,
-                                uint64_t *mask, void *scratch, cudaStream_t st);
-// Back to the resting state of the fused kernel's grid barrier (after a
-// timeout left it inconsistent); the device must be idle.
-cudaError_t reset_decode_sync();
 
 // Scratch carve-up of the tensor-core path.
 struct TcPlan {
@@ -355,5 +340,11 @@ cudaError_t launch_tc_logits_tau(const FwdShape &s, const DeviceInfo &dev, const
 cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint16_t *act,
                            const void *Wd, void *y, int ksplit, cudaStream_t st,
                            bool f32_out = false);
+// C[M][ldc] (=, or += when accumulate) A B on the tensor cores: bf16
+// operands, float32 out.  A [M][K] (row stride lda), or [K][M] when a_mn; B
+// [N][K] (ldb), or [K][N] when b_mn.  N % 64 == 0; a_mn needs b_mn.
+cudaError_t launch_tc_gemm_f32(const DeviceInfo &dev, int M, int N, int K, const void *A,
+                               int lda, bool a_mn, const void *B, int ldb, bool b_mn, float *C,
+                               int ldc, bool accumulate, cudaStream_t st);
 
 }  // namespace sfn

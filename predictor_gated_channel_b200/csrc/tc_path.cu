@@ -59,7 +59,13 @@ enum : int {
   kEpiTopk = 2,
   kEpiGateUp = 3,
   kEpiDown = 4,
-  kEpiDense4x = 5  // gate/up GEMM of the post-hoc amplitude top-k comparison
+  kEpiDense4x = 5,  // gate/up GEMM of the post-hoc amplitude top-k comparison
+  // plain float32 products C (=, +=) A B of the backward; the suffix gives
+  // the storage of A and B: K = K-major ([M][K], [N][K]), M = MN-major
+  // ([K][M], [K][N])
+  kEpiF32KK = 6,
+  kEpiF32KM = 7,
+  kEpiF32MM = 8
 };
 
 struct TcParams {
@@ -86,20 +92,23 @@ struct TcParams {
                           // into out ([T][ld_out]); sig may then be null
   bool b_once;            // the B operand (weights) is read once (one token tile): its
                           // loads carry an evict-first L2 policy
+  bool accumulate;        // float32 products: add to the output instead of overwriting
   unsigned *err;
 };
 
 template <int kEpi>
 struct EpiTraits {
   static constexpr int kNumA = (kEpi == kEpiLogits || kEpi == kEpiTopk) ? 2 : 1;
-  static constexpr bool kBMnMajor = (kEpi == kEpiDown);
+  static constexpr bool kF32 = (kEpi == kEpiF32KK || kEpi == kEpiF32KM || kEpi == kEpiF32MM);
+  static constexpr bool kAMnMajor = (kEpi == kEpiF32MM);
+  static constexpr bool kBMnMajor = (kEpi == kEpiDown || kEpi == kEpiF32KM || kEpi == kEpiF32MM);
   static constexpr bool kGateUpB = (kEpi == kEpiGateUp || kEpi == kEpiDense4x);
   // epilogue warps: two per TMEM lane quadrant for the top-k (its sorting
   // networks, not the MMAs, bound that GEMM) and for gate/up and down (with
   // one tile per CTA at few tokens, their epilogue is a serial tail after
   // the mainloop), splitting the tile's banks or column chunks
   static constexpr int kEpiWarps =
-      (kEpi == kEpiTopk || kEpi == kEpiGateUp || kEpi == kEpiDown) ? 8 : 4;
+      (kEpi == kEpiTopk || kEpi == kEpiGateUp || kEpi == kEpiDown || kF32) ? 8 : 4;
   static constexpr int kThreads = (2 + kEpiWarps) * 32;
 };
 
@@ -307,10 +316,10 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           if (Tr::kGateUpB) {
             load_b(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
             load_b(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
-          } else if (kEpi == kEpiDown) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              load_b(b + q * 8192, &tB, nb * kAccCols + q * 64, kb * kBK, &full[s]);
+          } else if (Tr::kBMnMajor) {
+            // [K][N] storage: bn/64 boxes of 64 N-elements x 64 K-rows
+            for (int q = 0; q < p.bn / 64; ++q)
+              load_b(b + q * 8192, &tB, nb * p.bn + q * 64, kb * kBK, &full[s]);
           } else {
             load_b(b, &tB, kb * kBK, nb * p.bn, &full[s]);
           }
@@ -343,7 +352,13 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
             unsigned char *a = smem + (size_t)s * p.stage_bytes;
             const bool fresh = !kOnce || (int)it >= pre;  // weights not issued yet
             if (fresh) mbar_arrive_expect_tx(&full[s], p.tx_bytes);
-            tma_load_2d(a, &tA, kb * kBK, mb * kBM, &full[s]);
+            if (Tr::kAMnMajor) {
+              // [K][M] storage: two boxes of 64 M-elements x 64 K-rows
+              tma_load_2d(a, &tA, mb * kBM, kb * kBK, &full[s]);
+              tma_load_2d(a + 8192, &tA, mb * kBM + 64, kb * kBK, &full[s]);
+            } else {
+              tma_load_2d(a, &tA, kb * kBK, mb * kBM, &full[s]);
+            }
             if (Tr::kNumA == 2)
               tma_load_2d(a + p.a_tile_bytes, &tA, p.r + kb * kBK, mb * kBM, &full[s]);
             if (fresh) issue_b(s, kb, nb);
@@ -386,14 +401,18 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           tc_fence_after();
           const unsigned char *a = smem + (size_t)s * p.stage_bytes;
           const unsigned char *b = a + Tr::kNumA * p.a_tile_bytes;
-          const uint64_t adesc = desc_kmajor_sw128(a);
+          const uint64_t adesc =
+              Tr::kAMnMajor ? desc_mnmajor_sw128(a, 8192) : desc_kmajor_sw128(a);
           const uint64_t adesc2 = desc_kmajor_sw128(a + p.a_tile_bytes);
           const uint64_t bdesc =
               Tr::kBMnMajor ? desc_mnmajor_sw128(b, 8192) : desc_kmajor_sw128(b);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
+            // along K: 16 elements = 32 bytes (K-major) or 16 rows of 128
+            // bytes (MN-major), in units of 16 bytes
+            const uint64_t aoff = Tr::kAMnMajor ? (uint64_t)(kk * 2048 >> 4) : (uint64_t)(kk * 2);
             const uint64_t boff = Tr::kBMnMajor ? (uint64_t)(kk * 2048 >> 4) : (uint64_t)(kk * 2);
-            umma_f16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + boff, p.idesc,
+            umma_f16(d_tmem, adesc + aoff, bdesc + boff, p.idesc,
                      (kb > kb0 || kk > 0) ? 1u : 0u);
             if (Tr::kNumA == 2) umma_f16(d_tmem, adesc2 + (uint64_t)(kk * 2), bdesc + boff, p.idesc, 1u);
           }
@@ -448,12 +467,33 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
             }
           }
         }
-      } else if (kEpi == kEpiLogits || kEpi == kEpiDown || kEpi == kEpiHSplit) {
+      } else if (kEpi == kEpiLogits || kEpi == kEpiDown || kEpi == kEpiHSplit || Tr::kF32) {
         for (int c0 = 32 * half_id; c0 < p.bn; c0 += 32 * (Tr::kEpiWarps / 4)) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + c0, v);
           tmem_ld_wait();
-          if (valid) {
+          if (valid && Tr::kF32) {
+            // C (=, +=) A B, float32 [M][ld_out]
+            float *dst = reinterpret_cast<float *>(p.out) + t * p.ld_out + nb * p.bn + c0;
+            if (p.accumulate) {
+              float4 o[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o[i] = reinterpret_cast<const float4 *>(dst)[i];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                o[i].x += __uint_as_float(v[4 * i]);
+                o[i].y += __uint_as_float(v[4 * i + 1]);
+                o[i].z += __uint_as_float(v[4 * i + 2]);
+                o[i].w += __uint_as_float(v[4 * i + 3]);
+                reinterpret_cast<float4 *>(dst)[i] = o[i];
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                reinterpret_cast<uint4 *>(dst)[i] =
+                    make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+          } else if (valid) {
             const int col = nb * p.bn + c0;
             if (kEpi != kEpiDown || p.ksplit > 1 || p.f32_out) {
               // fp32 logits, or fp32 partial sums [T][ksplit][ld_out]
@@ -663,12 +703,13 @@ bool encoder() {
   return g_encode != nullptr;
 }
 
-// Row-major bf16 matrix [outer][inner], box {box_inner, box_outer}, 128-byte
-// swizzle, zero fill outside.
+// Row-major bf16 matrix [outer][inner] with rows `stride` elements apart
+// (0: inner), box {box_inner, box_outer}, 128-byte swizzle, zero fill
+// outside.
 bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer, uint64_t stride = 0) {
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {(stride ? stride : inner) * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
@@ -681,7 +722,7 @@ template <int kEpi>
 cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtensorMap &tB2,
                       TcParams p, int num_sms, cudaStream_t st) {
   using Tr = EpiTraits<kEpi>;
-  const uint32_t b_bytes = (kEpi == kEpiDown) ? 32768u : (uint32_t)p.bn * 128u;
+  const uint32_t b_bytes = (uint32_t)p.bn * 128u;  // 64 K-rows of bn elements
   // A tiles hold only the token rows loaded; the MMA still reads kBM rows
   // (kTileA bytes) from each A tile start, which may run past the stage: a
   // tail of kTileA bytes keeps every such read inside the allocation
@@ -696,7 +737,7 @@ cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtens
   p.stages = (int)(((size_t)kMaxDynSmem - fixed) / p.stage_bytes);
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return cudaErrorInvalidValue;
-  p.idesc = idesc_bf16_f32(kBM, p.bn, Tr::kBMnMajor);
+  p.idesc = idesc_bf16_f32(kBM, p.bn, Tr::kBMnMajor, Tr::kAMnMajor);
   const size_t smem = fixed + (size_t)p.stages * p.stage_bytes;
   if ((2 * p.stages + 5) * 8 + 4 > 256) return cudaErrorInvalidValue;
   auto kern = k_tc_gemm<kEpi>;
@@ -944,6 +985,39 @@ cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint1
   p.ld_out = s.d;
   p.f32_out = f32_out;
   return launch_tc<kEpiDown>(mAct, mD, mD, p, dev.num_sms, st);
+}
+
+// C[M][ldc] (=, or += when accumulate) A B: bf16 operands, float32
+// accumulation and output.  A is [M][K] (lda elements per row), or [K][M]
+// when a_mn; B is [N][K] (ldb), or [K][N] when b_mn.  N must be a multiple of
+// 64; M and K are arbitrary (the loads zero-fill past them).
+cudaError_t launch_tc_gemm_f32(const DeviceInfo &dev, int M, int N, int K, const void *A,
+                               int lda, bool a_mn, const void *B, int ldb, bool b_mn, float *C,
+                               int ldc, bool accumulate, cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  if (M <= 0 || K <= 0 || N <= 0 || N % 64 != 0 || (a_mn && !b_mn)) return cudaErrorInvalidValue;
+  const int tiles_m = (M + kBM - 1) / kBM;
+  const int bn = pick_bn(tiles_m, N, {256, 128, 64}, dev.num_sms);
+  CUtensorMap mA, mB;
+  const bool okA = a_mn ? make_map(&mA, A, (uint64_t)M, (uint64_t)K, 64, 64, (uint64_t)lda)
+                        : make_map(&mA, A, (uint64_t)K, (uint64_t)M, 64, kBM, (uint64_t)lda);
+  const bool okB = b_mn ? make_map(&mB, B, (uint64_t)N, (uint64_t)K, 64, 64, (uint64_t)ldb)
+                        : make_map(&mB, B, (uint64_t)K, (uint64_t)N, 64, bn, (uint64_t)ldb);
+  if (!okA || !okB) return cudaErrorInvalidValue;
+  TcParams p{};
+  p.T = M;
+  p.err = dev.err;
+  p.tiles_m = tiles_m;
+  p.tiles_n = N / bn;
+  p.k_blocks = (K + kBK - 1) / kBK;
+  p.ksplit = 1;
+  p.bn = bn;
+  p.out = C;
+  p.ld_out = ldc;
+  p.accumulate = accumulate;
+  if (a_mn) return launch_tc<kEpiF32MM>(mA, mB, mB, p, dev.num_sms, st);
+  if (b_mn) return launch_tc<kEpiF32KM>(mA, mB, mB, p, dev.num_sms, st);
+  return launch_tc<kEpiF32KK>(mA, mB, mB, p, dev.num_sms, st);
 }
 
 }  // namespace sfn

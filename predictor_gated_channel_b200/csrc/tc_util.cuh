@@ -12,6 +12,9 @@
 //   instruction descriptor (32 bit): D format [4,6) (1 = f32), A format
 //   [7,10) and B format [10,13) (1 = bf16), A major [15], B major [16]
 //   (0 = K-major, 1 = MN-major), N >> 3 [17,23), M >> 4 [24,29).
+//   An MN-major operand tile is read through the same descriptor format as
+//   desc_mnmajor_sw128 below (64-element MN blocks `leading byte offset`
+//   apart, 8-row K groups 1024 B apart).
 #pragma once
 
 #include <cuda.h>
@@ -143,11 +146,13 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(const void *smem_tile,
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor: bf16 x bf16 -> f32, M x N, A K-major, B K- or
+// Instruction descriptor: bf16 x bf16 -> f32, M x N, A and B each K- or
 // MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major,
+                                                      bool a_mn_major = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace sfn

@@ -4,8 +4,20 @@ fp64 oracle, through the C ABI.
 The oracle runs on the GPU's own mask (a mask flip allowed by the forward's
 rule changes which channels carry gradient, so it is not counted as error);
 the mask itself is checked with the forward's rule.  Gradients come from bf16
-GEMM operands with float32 accumulation, so each is compared as
-max |gpu - oracle| / max |oracle| <= 2e-2, the bf16 tolerance of the forward.
+GEMM operands with float32 accumulation, so each is compared row by row, like
+the forward's y:
+
+    max |gpu - oracle| over a row <= 2e-2 * max(max |oracle row|, 1e-4 * max |oracle|)
+
+(2e-2 is the bf16 tolerance of the forward), and a row the oracle gives as
+exactly zero (a channel no token keeps, in dWg, dWu, dWd) must be exactly
+zero.  The floor covers rows that are small only because a factor of theirs
+nearly cancels: in the full-width layer, g_j = W_gate[j] . x can be 1e-4 while
+its terms sum to 40 in magnitude, and float32 accumulation in any order then
+leaves about 1e-2 relative error in g_j and in the whole weight-gradient row
+built from it.  Below 1e-4 of the matrix's largest row the check is absolute,
+at 2e-6 of that row -- ten thousand times tighter than one bound for the
+whole matrix.
 """
 import math
 
@@ -58,6 +70,22 @@ def _run(wl, host, dev, T, bank, k, temp, want=NAMES):
     return x, dy, out
 
 
+ROW_FLOOR = 1e-4
+
+
+def _check_rows(name, g, ref):
+    """Per-row error of a gradient matrix (see the module doc)."""
+    assert np.isfinite(g).all(), name
+    scale = np.abs(ref).max(axis=1)
+    err = np.abs(g - ref).max(axis=1)
+    zero = scale == 0
+    assert (err[zero] == 0).all(), f"{name}: rows the oracle gives as zero are not zero"
+    rel = err[~zero] / np.maximum(scale[~zero], ROW_FLOOR * scale.max())
+    worst = int(np.argmax(rel)) if len(rel) else 0
+    assert not len(rel) or rel.max() <= GRAD_TOL, (
+        f"{name}: row {np.flatnonzero(~zero)[worst]} relative error {rel.max():.3g}")
+
+
 def _check(wl, host, dev, T, bank, k, temp):
     x, dy, out = _run(wl, host, dev, T, bank, k, temp)
     gm = parity.to_u64(out["mask"])
@@ -65,11 +93,7 @@ def _check(wl, host, dev, T, bank, k, temp):
     ref = oracle.backward(x, host["A"], host["B"], host["Wg"], host["Wu"], host["Wd"], dy,
                           bank, k, temp, mask=gm)
     for n in NAMES:
-        g = out[n].cpu().numpy().astype(np.float64)
-        assert np.isfinite(g).all(), n
-        scale = np.abs(ref[n]).max()
-        err = np.abs(g - ref[n]).max() / max(scale, 1e-30)
-        assert err <= GRAD_TOL, f"{n}: max error {err:.3g} of max |oracle| {scale:.3g}"
+        _check_rows(n, out[n].cpu().numpy().astype(np.float64), ref[n])
     errs = np.zeros(1, np.int32)
     _capi.check(_capi.lib().sfn_device_errors(errs.ctypes.data, 1), "sfn_device_errors")
     assert errs[0] == 0
@@ -80,6 +104,8 @@ def _check(wl, host, dev, T, bank, k, temp):
     (5, 64, 16, 0.5),    # logits on the CUDA-core kernels
     (33, 16, 4, 0.3),    # bank 16: CUDA-core logits
     (20, 64, 64, 1.0),   # k = bank: no threshold, no surrogate term
+    (130, 64, 16, 0.5),  # two token tiles; the K = T contractions end mid-block
+    (300, 64, 16, 1.0),  # three token tiles, ragged in M and in K
 ])
 def test_backward_small(T, bank, k, temp):
     wl = SMALL.with_(bank=bank, k=k)

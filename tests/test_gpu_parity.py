@@ -223,10 +223,11 @@ def test_outputs_do_not_spill(full_layer):
 
 
 def test_launch_counter_counts_kernels(full_layer):
-    """One token: the single fused kernel; two tokens: the four few-token
-    kernels."""
+    """Few tokens: h, logits + top-k, and gate/up/down with the final sum in
+    one cooperative launch; many: the tensor path (h, its split-K sum,
+    logits + top-k, gate/up, down, its split-K sum at 64 tokens)."""
     wl, host, dev = full_layer
-    for T, n in ((1, 1), (2, 4)):
+    for T, n in ((1, 3), (2, 3), (64, 6)):
         x = make_tokens(wl, T=T).to(DEV)
         c0 = sfn.kernel_launch_count()
         _run_forward(dev, x, 64, 16)
@@ -302,14 +303,12 @@ def _bf16_dev(a):
     return torch.from_numpy(a).to(torch.bfloat16).to(DEV)
 
 
-@pytest.mark.parametrize("T,path", [(1, "cuda_core"), (3, "cuda_core"), (5, "cuda_core"),
-                                    (1, "decode_fused")])
+@pytest.mark.parametrize("T,path", [(1, "cuda_core"), (3, "cuda_core"), (5, "cuda_core")])
 @pytest.mark.parametrize("bank,k", [(64, 1), (64, 4), (64, 16), (64, 20), (64, 63), (48, 17),
                                     (32, 5)])
 def test_cuda_core_topk_exact_ties(T, path, bank, k):
-    """The few-token kernels rank each bank inside their logits stage (the
-    four-kernel path and the one-token fused kernel each have their own,
-    beside the standalone top-k and the tensor-core epilogue).  Fed
+    """The few-token kernels rank each bank inside their logits kernel (a
+    third top-k, beside the standalone one and the tensor-core epilogue).  Fed
     exact-integer logits with ties everywhere, the mask equals the oracle's
     bit for bit (ties to the lower channel), for k below, at and above 16,
     and for banks narrower than 64 (whose order-key rows are padded)."""
@@ -323,42 +322,41 @@ def test_cuda_core_topk_exact_ties(T, path, bank, k):
     assert np.array_equal(parity.to_u64(mask), oracle.bank_topk(p, bank, k))
 
 
-@pytest.mark.parametrize("seed,k", [(0, 16), (1, 16), (2, 1), (3, 63), (4, 64)])
-def test_decode_fused_full_width(seed, k, full_layer):
-    """The one-token cooperative kernel on the full-width layer against the
-    oracle (mask rule and y tolerance), for k below, at and above 16 and the
-    dense k = bank case."""
+@pytest.mark.parametrize("T,k", [(1, 16), (1, 1), (1, 63), (1, 64), (2, 16), (4, 16), (5, 16)])
+def test_few_token_cooperative_sum(T, k, full_layer):
+    """The few-token gate/up/down kernel that also sums its partial rows
+    after a grid-wide barrier (one cooperative launch) against the oracle,
+    for k below, at and above 16, k = bank, and 1 to 5 tokens."""
     wl, host, dev = full_layer
-    x = make_tokens(wl, T=1, seed=500 + seed)
+    x = make_tokens(wl, T=T, seed=500 + 10 * T + k)
     y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
-                                     dev["Wd"], k=k, path="decode_fused")
+                                     dev["Wd"], k=k, path="cuda_core")
     torch.cuda.synchronize()
     _check_forward(host, x, y, mask, 64, k, "bf16")
 
 
-def test_decode_fused_many_calls_bit_identical(full_layer):
-    """Sixty launches in a row on one stream: every launch passes both grid
-    barriers (whose state carries from launch to launch) and reproduces the
-    first result bit for bit; the automatic choice at one token is this
-    kernel, and a one-token bank shard (float32 partial y) sums to the layer."""
+def test_cooperative_sum_many_calls_bit_identical(full_layer):
+    """Sixty calls in a row on one stream: every call passes the grid barrier
+    (whose state carries from launch to launch) and reproduces the first
+    result bit for bit; a one-token bank shard (float32 partial y, the
+    cooperative sum writing float32) sums to the layer."""
     wl, host, dev = full_layer
     xs = [make_tokens(wl, T=1, seed=600 + i).to(DEV) for i in range(3)]
     first = [_run_forward(dev, x, 64, 16) for x in xs]
     c0 = sfn.kernel_launch_count()
     outs = [sfn.sparse_ffn_forward(xs[i % 3], dev["A"], dev["B"], dev["Wg"], dev["Wu"],
-                                   dev["Wd"], path="decode_fused") for i in range(60)]
+                                   dev["Wd"]) for i in range(60)]
     torch.cuda.synchronize()
-    assert sfn.kernel_launch_count() - c0 == 60  # one kernel per call
+    assert sfn.kernel_launch_count() - c0 == 3 * 60  # h, logits + top-k, gate/up/down + sum
     for i, (y, m) in enumerate(outs):
         assert torch.equal(y, first[i % 3][0]) and torch.equal(m, first[i % 3][1]), i
-    # bank shards at one token: float32 partial outputs sum to the layer
     total = torch.zeros((1, wl.d), dtype=torch.float32, device=DEV)
     for rank in range(2):
         b0, b1 = sfn.bank_shard(wl.n_banks, rank, 2)
         rows = slice(b0 * wl.bank, b1 * wl.bank)
         yp, _ = sfn.sparse_ffn_forward_partial(xs[0], dev["A"], dev["B"][rows],
                                                dev["Wg"][rows], dev["Wu"][rows],
-                                               dev["Wd"][rows], path="decode_fused")
+                                               dev["Wd"][rows])
         total += yp
     torch.cuda.synchronize()
     ref = first[0][0].float()
