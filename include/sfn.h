@@ -207,22 +207,13 @@ sfn_status sfn_sparse_ffn_forward_static(const void *x, const void *A, const voi
  * (within rounding; the mask may differ only at exact-threshold ties of the
  * differently rounded logits).
  *   SFN_PATH_CUDA_CORE  gather kernels that read only the kept rows (few
- *                       tokens: every T, any bank <= 64, bf16 or f32); when
- *                       all of the call's gate/up/down CTAs fit the device at
- *                       once (T <= 5 on a B200), the final sum of their
- *                       partial rows runs in the same cooperative launch
- *                       after a grid-wide barrier, else in a kernel of its
- *                       own;
+ *                       tokens: every T, any bank <= 64, bf16 or f32);
  *   SFN_PATH_TENSOR     tcgen05 tensor-core GEMMs over 128-token tiles with
  *                       the top-k and the sigma(p) g u mask fused into their
  *                       epilogues (bf16, bank 64, d and d_i multiples of
  *                       256, r a multiple of 64 up to 512);
  *   SFN_PATH_AUTO       the tensor path from T >= 6 when the shape allows
  *                       it, the CUDA-core path otherwise.
- * The cooperative launch's barrier state lives in the library and is shared
- * by its launches on a device; two of them never run at the same time (each
- * takes one CTA on every SM it uses, and cooperative grids are placed only
- * when all their CTAs fit), so concurrent calls on other streams stay safe.
  */
 typedef enum sfn_path {
   SFN_PATH_AUTO = 0,
@@ -339,9 +330,7 @@ sfn_status sfn_sparse_ffn_forward_f32_ws(const float *x, const float *A, const f
 enum {
   SFN_STAGE_PRED_H = 0,       /* h = A x                                */
   SFN_STAGE_LOGITS_TOPK = 1,  /* p = B h, bank top-k, sigma(p) of kept  */
-  SFN_STAGE_FFN = 2,          /* kept gate/up/down rows -> partial y
-                                 (and y itself, when summed in the same
-                                 cooperative launch)                    */
+  SFN_STAGE_FFN = 2,          /* kept gate/up/down rows -> partial y    */
   SFN_STAGE_REDUCE = 3,       /* partial rows -> y (few tokens)         */
   SFN_STAGE_BANK_TOPK = 4,    /* standalone top-k on given logits       */
   SFN_STAGE_TC_H = 5,         /* tensor cores: h = A x, split hi/lo     */
@@ -362,9 +351,7 @@ sfn_status sfn_timing_begin(void);
  * two seconds, or a failed index check, sets a bit here and the kernel
  * returns early (its outputs are then invalid).  Bits: 1 = a bounded wait
  * timed out, 2 = an index check failed.  This call synchronises the device,
- * writes the word to *bits and, if `clear`, resets it to 0 (and the
- * grid-barrier state of the cooperative gate/up/down kernel, which a wait
- * that gave up may have left mid-episode).  The word's
+ * writes the word to *bits and, if `clear`, resets it to 0.  The word's
  * address is looked up once per device and cached; cudaDeviceReset
  * invalidates it (and every other per-device cache of the library).
  */

@@ -340,24 +340,16 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
       e = timed(SFN_STAGE_LOGITS_TOPK, st, [&] {
         return launch_logits_topk(s, p.tt_p, h, B, nullptr, mask, sel_idx, sel_sig, dev.err, st);
       });
-    if (ffn_sum_ok(s, p.cpt, dev)) {
-      // gate/up/down and the sum of the partial rows in one cooperative launch
-      if (e == cudaSuccess)
-        e = timed(SFN_STAGE_FFN, st, [&] {
-          return launch_ffn_sum(s, p.cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, y, y_f32,
-                                dev.err, st);
-        });
-    } else {
-      if (e == cudaSuccess)
-        e = timed(SFN_STAGE_FFN, st, [&] {
-          return launch_ffn(s, p.cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, dev.err, st);
-        });
-      if (e == cudaSuccess)
-        e = timed(SFN_STAGE_REDUCE, st, [&] {
-          return launch_reduce_partials(s, p.cpt, partial, y, st,
-                                        y_f32 ? ReduceOut::kYF32 : ReduceOut::kY);
-        });
-    }
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_FFN, st, [&] {
+        return launch_ffn(s, p.cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, dev.err, st);
+      });
+    if (e == cudaSuccess)
+      e = timed(SFN_STAGE_REDUCE, st,
+                [&] {
+                  return launch_reduce_partials(s, p.cpt, partial, y, st,
+                                                y_f32 ? ReduceOut::kYF32 : ReduceOut::kY);
+                });
   }
   if (own_ws) {
     cudaError_t ef = cudaFreeAsync(ws, st);
@@ -540,14 +532,8 @@ sfn_status sfn_device_errors(unsigned *bits, int clear) {
   unsigned v = 0;
   if (cudaMemcpy(&v, dev.err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
     return cuda_status(cudaErrorUnknown);
-  if (clear && v != 0) {
-    if (cudaMemset(dev.err, 0, sizeof v) != cudaSuccess) return cuda_status(cudaErrorUnknown);
-    // a wait that gave up may have left the cooperative gate/up/down
-    // kernel's grid barrier mid-episode: back to its resting state (the
-    // device is idle)
-    if (reset_grid_sync() != cudaSuccess) return cuda_status(cudaErrorUnknown);
-    if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaErrorUnknown);
-  }
+  if (clear && v != 0 && cudaMemset(dev.err, 0, sizeof v) != cudaSuccess)
+    return cuda_status(cudaErrorUnknown);
   if (bits) *bits = v;
   return SFN_OK;
 }

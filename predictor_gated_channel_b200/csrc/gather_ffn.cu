@@ -16,10 +16,6 @@
 //                      down warp owns one eighth of the output columns in
 //                      registers and accumulates a * Wd[j, cols] over the
 //                      slots in order.  The CTA writes one fp32 partial row.
-//   k_ffn_sum          k_ffn_ring and the sum of its partial rows in one
-//                      cooperative launch: after the ring, a grid-wide
-//                      barrier, then every CTA sums its share of the outputs
-//                      (used when the grid fits the device at once).
 //   k_reduce_partials  y[t] = sum of the token's partial rows in a fixed
 //                      order, rounded to the output type.  Also the tensor
 //                      path's split-K sums (fp32 partials of h and of y).
@@ -27,9 +23,6 @@
 //                      columns, no shared memory.
 // Only the kept rows of Wg, Wu and Wd are read, each once per token; all sums
 // run in a fixed order, so results are bit-reproducible.
-#include <mutex>
-#include <vector>
-
 #include "async_util.cuh"
 #include "sfn_internal.cuh"
 
@@ -69,34 +62,15 @@ __host__ __device__ inline RingLayout ring_layout(int d, int elt_bytes) {
   return L;
 }
 
-// Four consecutive outputs v at out[i .. i + 4): kOut 0 float32, 1 bf16.
-template <int kOut>
-__device__ __forceinline__ void store_quad(void *out, int64_t i, float4 v) {
-  if (kOut == 0) {
-    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + i) = v;
-  } else {
-    uint2 o;
-    o.x = (uint32_t)f32_to_bf16_bits(v.x) | ((uint32_t)f32_to_bf16_bits(v.y) << 16);
-    o.y = (uint32_t)f32_to_bf16_bits(v.z) | ((uint32_t)f32_to_bf16_bits(v.w) << 16);
-    *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(out) + i) = o;
-  }
-}
-
-// The ring: this CTA's partial row of y.  blockDim.x = (stages + kDownWarps
-// + 1) * 32: warps [0, S) gate/up, [S, S + 8) down, the last warp produces.
-// blockIdx.x = t * cpt + c.  Every thread returns from it (no thread leaves
-// the kernel inside), so a caller may go on with block-wide steps.
-// kReleaseEarly: let the stream's next kernel start right after the
-// dependency wait (else the caller releases it later).
-template <class E, bool kReleaseEarly>
-__device__ __forceinline__ void ffn_ring(unsigned char *smem, const char *__restrict__ x,
-                                         const int *__restrict__ sel_idx,
-                                         const float *__restrict__ sel_sig,
-                                         const char *__restrict__ Wg,
-                                         const char *__restrict__ Wu,
-                                         const char *__restrict__ Wd,
-                                         float *__restrict__ partial, int d_s, int d, int cpt,
-                                         unsigned *err) {
+// blockDim.x = (stages + kDownWarps + 1) * 32: warps [0, S) gate/up,
+// [S, S + 8) down, the last warp produces.  blockIdx.x = t * cpt + c.
+template <class E>
+__global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
+    k_ffn_ring(const char *__restrict__ x, const int *__restrict__ sel_idx,
+               const float *__restrict__ sel_sig, const char *__restrict__ Wg,
+               const char *__restrict__ Wu, const char *__restrict__ Wd,
+               float *__restrict__ partial, int d_s, int d, int cpt, unsigned *err) {
+  extern __shared__ __align__(128) unsigned char smem[];
   const RingLayout L = ring_layout(d, E::kBytes);
   const int S = L.stages;
   unsigned char *gu_ring = smem + L.off_gu;  // [S][2][row]
@@ -127,7 +101,7 @@ __device__ __forceinline__ void ffn_ring(unsigned char *smem, const char *__rest
     fence_barrier_init();
   }
   pdl_wait();  // sel_idx and sel_sig come from the previous kernel
-  if (kReleaseEarly) pdl_launch_dependents();
+  pdl_launch_dependents();
   // stage this CTA's kept channel ids, their sigma(p) and the token's x;
   // each thread issues its loads before its stores (one round trip)
   const uint32_t row = L.row_bytes;
@@ -255,145 +229,6 @@ __device__ __forceinline__ void ffn_ring(unsigned char *smem, const char *__rest
   }
 }
 
-template <class E>
-__global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
-    k_ffn_ring(const char *__restrict__ x, const int *__restrict__ sel_idx,
-               const float *__restrict__ sel_sig, const char *__restrict__ Wg,
-               const char *__restrict__ Wu, const char *__restrict__ Wd,
-               float *__restrict__ partial, int d_s, int d, int cpt, unsigned *err) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  ffn_ring<E, true>(smem, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, d_s, d, cpt, err);
-}
-
-// Grid barrier state of k_ffn_sum: the number of CTA arrivals since the
-// library was loaded (or since reset_grid_sync), never reset by a kernel.
-// Episode e of a grid of G CTAs is complete when the count reaches
-// (e + 1) * G; a 64-bit count does not wrap.  k_ffn_sum grids are
-// cooperative and fill every SM, so two never run at the same time.
-struct GridSync {
-  unsigned long long count;
-  unsigned long long pad[15];
-};
-__device__ GridSync g_ffn_sync;
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Grid-wide barrier over gridDim.x co-resident CTAs: the writes of every
-// thread of every CTA before it are visible to every thread after it.  One
-// release add per CTA (its return value gives the episode), then acquire
-// polling; bounded (false and kDevErrWaitTimeout if the others do not come).
-__device__ bool grid_sync(unsigned *err, int *s_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    unsigned long long old;
-    __threadfence();
-    asm volatile("atom.add.release.gpu.global.u64 %0, [%1], 1;"
-                 : "=l"(old)
-                 : "l"(&g_ffn_sync.count)
-                 : "memory");
-    const unsigned long long G = gridDim.x;
-    const unsigned long long target = (old / G + 1) * G;
-    if (old + 1 != target) {
-      const long long t0 = clock64();
-      while (ld_acquire_u64(&g_ffn_sync.count) < target) {
-        if (clock64() - t0 > kWaitLimitCycles) {
-          report_error(err, kDevErrWaitTimeout);
-          ok = 0;
-          break;
-        }
-        __nanosleep(32);
-      }
-    }
-    *s_flag = ok;
-  }
-  __syncthreads();
-  return *s_flag != 0;
-}
-
-constexpr int kSumBatch = 5;  // partial-row loads in flight per thread
-
-// The few-token gate/up/down with the final sum in the same launch
-// (cooperative: every CTA resident).  After its ring, every CTA has written
-// its partial row; a grid barrier; then CTA b sums the partial rows of its
-// share of the T x d outputs, quads [b Q / G, (b + 1) Q / G) of the Q = T d / 4:
-// thread (g, qi), g < 32, adds partial rows g, g + 32, ... of quad qi, then
-// 4 x 8 threads add 8 groups each and 8 threads the 4 parts -- a fixed order,
-// so the result is bit-reproducible.  The stream's next kernel is released
-// after the barrier, so that its prologue (the next call's L2 prefetch of the
-// predictor's B) falls in this sum's idle DRAM time, not in the row stream.
-// kOut: 0 float32 y, 1 bf16 y.
-template <class E, int kOut>
-__global__ void __launch_bounds__((kMaxStages + kDownWarps + 1) * 32, 1)
-    k_ffn_sum(const char *__restrict__ x, const int *__restrict__ sel_idx,
-              const float *__restrict__ sel_sig, const char *__restrict__ Wg,
-              const char *__restrict__ Wu, const char *__restrict__ Wd,
-              float *__restrict__ partial, void *__restrict__ y, int d_s, int d, int cpt,
-              int T, unsigned *err) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_flag;
-  ffn_ring<E, false>(smem, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, d_s, d, cpt, err);
-  const bool ok = grid_sync(err, &s_flag);
-  pdl_launch_dependents();
-  if (!ok) return;
-  const int G = gridDim.x, b = blockIdx.x;
-  const int nq_t = d / 4;
-  const int64_t nq = (int64_t)T * nq_t;
-  const int64_t q_a = nq * b / G, q_b = nq * (b + 1) / G;
-  float4 *red = reinterpret_cast<float4 *>(smem);  // [32][8], the ring is done
-  float4 *red2 = red + 32 * 8;                     // [4][8]
-  const int qi = threadIdx.x & 7, g = threadIdx.x >> 3;
-  auto add4 = [](float4 &a, const float4 &v) {
-    a.x += v.x;
-    a.y += v.y;
-    a.z += v.z;
-    a.w += v.w;
-  };
-  for (int64_t qb0 = q_a; qb0 < q_b; qb0 += 8) {
-    const int64_t q = qb0 + qi;
-    const int64_t t = q / nq_t;
-    const int col = (int)(q - t * nq_t) * 4;
-    if (g < 32) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (q < q_b) {
-        const float *src = partial + t * cpt * (int64_t)d + col;
-        for (int j0 = g; j0 < cpt; j0 += 32 * kSumBatch) {
-          float4 v[kSumBatch];
-#pragma unroll
-          for (int u = 0; u < kSumBatch; ++u) {
-            const int j = j0 + 32 * u;
-            v[u] = j < cpt ? __ldcg(reinterpret_cast<const float4 *>(src + (int64_t)j * d))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-          for (int u = 0; u < kSumBatch; ++u) add4(acc, v[u]);
-        }
-      }
-      red[g * 8 + qi] = acc;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      const int part = threadIdx.x >> 3;
-      float4 v = red[(part * 8) * 8 + qi];
-#pragma unroll
-      for (int gg = 1; gg < 8; ++gg) add4(v, red[(part * 8 + gg) * 8 + qi]);
-      red2[part * 8 + qi] = v;
-    }
-    __syncthreads();
-    if (threadIdx.x < 8 && q < q_b) {
-      float4 v = red2[qi];
-#pragma unroll
-      for (int part = 1; part < 4; ++part) add4(v, red2[part * 8 + qi]);
-      store_quad<kOut>(y, t * d + col, v);
-    }
-    __syncthreads();
-  }
-}
-
 // out[t][c0 .. c0+C) = sum_{c < cpt} partial[t][c][c0 .. c0+C), summed in a
 // fixed order.  blockIdx.x = t * ceil(n / C) + slice.  Thread = (group g,
 // quad q), q fastest: group g sums partials c = g, g + G, ... (its loads
@@ -489,6 +324,19 @@ __global__ void __launch_bounds__(kReduceThreads) k_reduce_partials(
   }
 }
 
+// Four consecutive outputs v at out[i .. i + 4): kOut 0 float32, 1 bf16.
+template <int kOut>
+__device__ __forceinline__ void store_quad(void *out, int64_t i, float4 v) {
+  if (kOut == 0) {
+    *reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + i) = v;
+  } else {
+    uint2 o;
+    o.x = (uint32_t)f32_to_bf16_bits(v.x) | ((uint32_t)f32_to_bf16_bits(v.y) << 16);
+    o.y = (uint32_t)f32_to_bf16_bits(v.z) | ((uint32_t)f32_to_bf16_bits(v.w) << 16);
+    *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(out) + i) = o;
+  }
+}
+
 // Few partials (cpt <= kSmallCpt): one thread per four columns adds the cpt
 // partial rows in order 0, 1, ..., with its loads in flight together.  No
 // shared memory, so its CTAs fit beside a large-shared-memory kernel still
@@ -577,89 +425,6 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
                        float *partial, unsigned *err, cudaStream_t st) {
   if (s.bf16) return ffn_e<EltBF16>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, err, st);
   return ffn_e<EltF32>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, err, st);
-}
-
-namespace {
-template <class E, int kOut>
-cudaError_t ffn_sum_e(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
-                      const float *sel_sig, const void *Wg, const void *Wu, const void *Wd,
-                      float *partial, void *y, unsigned *err, cudaStream_t st) {
-  const RingLayout L = ring_layout(s.d, E::kBytes);
-  auto kern = k_ffn_sum<E, kOut>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), L.total);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(cpt * s.T));
-  cfg.blockDim = dim3((L.stages + kDownWarps + 1) * 32);
-  cfg.dynamicSmemBytes = L.total;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, (const char *)x, sel_idx, sel_sig, (const char *)Wg,
-                         (const char *)Wu, (const char *)Wd, partial, y, s.d_s, s.d, cpt,
-                         (int)s.T, err);
-  count_launches(1);
-  return e;
-}
-}  // namespace
-
-bool ffn_sum_ok(const FwdShape &s, int cpt, const DeviceInfo &dev) {
-  if (!ffn_shape_ok(s) || s.T < 1 || s.T * (int64_t)cpt > dev.num_sms) return false;
-  // one CTA per SM must be resident for every CTA of the grid: asked once
-  // per (device, element type, row length)
-  struct Known {
-    int device, elt, d;
-    bool ok;
-  };
-  static std::mutex mu;
-  static std::vector<Known> known;
-  const int elt = s.bf16 ? 2 : 4;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    for (const Known &k : known)
-      if (k.device == dev.device && k.elt == elt && k.d == s.d) return k.ok;
-  }
-  const RingLayout L = ring_layout(s.d, elt);
-  const void *kerns[2] = {
-      s.bf16 ? reinterpret_cast<const void *>(k_ffn_sum<EltBF16, 1>)
-             : reinterpret_cast<const void *>(k_ffn_sum<EltF32, 0>),
-      s.bf16 ? reinterpret_cast<const void *>(k_ffn_sum<EltBF16, 0>)
-             : reinterpret_cast<const void *>(k_ffn_sum<EltF32, 0>)};
-  bool ok = true;
-  for (const void *kern : kerns) {
-    int per_sm = 0;
-    if (ensure_smem_limit(kern, L.total) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &per_sm, kern, (L.stages + kDownWarps + 1) * 32, L.total) != cudaSuccess) {
-      cudaGetLastError();
-      ok = false;
-    }
-    ok = ok && per_sm >= 1;
-  }
-  std::lock_guard<std::mutex> lock(mu);
-  known.push_back({dev.device, elt, s.d, ok});
-  return ok;
-}
-
-cudaError_t launch_ffn_sum(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
-                           const float *sel_sig, const void *Wg, const void *Wu,
-                           const void *Wd, float *partial, void *y, bool y_f32, unsigned *err,
-                           cudaStream_t st) {
-  if (s.bf16 && !y_f32)
-    return ffn_sum_e<EltBF16, 1>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, y, err, st);
-  if (s.bf16)
-    return ffn_sum_e<EltBF16, 0>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, y, err, st);
-  return ffn_sum_e<EltF32, 0>(s, cpt, x, sel_idx, sel_sig, Wg, Wu, Wd, partial, y, err, st);
-}
-
-cudaError_t reset_grid_sync() {
-  void *addr = nullptr;
-  cudaError_t e = cudaGetSymbolAddress(&addr, g_ffn_sync);
-  if (e != cudaSuccess) return e;
-  return cudaMemset(addr, 0, sizeof(GridSync));
 }
 
 template <int C>

@@ -290,17 +290,7 @@ cudaError_t launch_ffn(const FwdShape &s, int cpt, const void *x, const int *sel
 // kYF32: y as float32 whatever the input type (partial outputs of a bank
 // shard, summed across devices before rounding).
 enum class ReduceOut { kY, kYF32, kSplitH };
-// The few-token gate/up/down with the final sum in the same cooperative
-// launch (k_ffn_sum, T * cpt CTAs, one per SM): y (bf16 or float32 per the
-// call) instead of partial rows for a separate sum.  ffn_sum_ok tells whether
-// the grid fits the device; reset_grid_sync returns its grid barrier to the
-// resting state after a wait gave up (the device must be idle).
-bool ffn_sum_ok(const FwdShape &s, int cpt, const DeviceInfo &dev);
-cudaError_t launch_ffn_sum(const FwdShape &s, int cpt, const void *x, const int *sel_idx,
-                           const float *sel_sig, const void *Wg, const void *Wu,
-                           const void *Wd, float *partial, void *y, bool y_f32, unsigned *err,
-                           cudaStream_t st);
-cudaError_t reset_grid_sync();
+
 cudaError_t launch_reduce_partials(const FwdShape &s, int cpt, const float *partial, void *y,
                                    cudaStream_t st, ReduceOut kind = ReduceOut::kY);
 

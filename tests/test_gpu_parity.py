@@ -223,11 +223,11 @@ def test_outputs_do_not_spill(full_layer):
 
 
 def test_launch_counter_counts_kernels(full_layer):
-    """Few tokens: h, logits + top-k, and gate/up/down with the final sum in
-    one cooperative launch; many: the tensor path (h, its split-K sum,
-    logits + top-k, gate/up, down, its split-K sum at 64 tokens)."""
+    """Few tokens: h, logits + top-k, gate/up/down, the sum of the partial
+    rows; many: the tensor path (h, its split-K sum, logits + top-k,
+    gate/up, down, its split-K sum at 64 tokens)."""
     wl, host, dev = full_layer
-    for T, n in ((1, 3), (2, 3), (64, 6)):
+    for T, n in ((1, 4), (2, 4), (64, 6)):
         x = make_tokens(wl, T=T).to(DEV)
         c0 = sfn.kernel_launch_count()
         _run_forward(dev, x, 64, 16)
@@ -323,10 +323,9 @@ def test_cuda_core_topk_exact_ties(T, path, bank, k):
 
 
 @pytest.mark.parametrize("T,k", [(1, 16), (1, 1), (1, 63), (1, 64), (2, 16), (4, 16), (5, 16)])
-def test_few_token_cooperative_sum(T, k, full_layer):
-    """The few-token gate/up/down kernel that also sums its partial rows
-    after a grid-wide barrier (one cooperative launch) against the oracle,
-    for k below, at and above 16, k = bank, and 1 to 5 tokens."""
+def test_few_token_path_k_variants(T, k, full_layer):
+    """The few-token kernels on the full-width layer against the oracle, for
+    k below, at and above 16, k = bank, and 1 to 5 tokens."""
     wl, host, dev = full_layer
     x = make_tokens(wl, T=T, seed=500 + 10 * T + k)
     y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
@@ -335,11 +334,11 @@ def test_few_token_cooperative_sum(T, k, full_layer):
     _check_forward(host, x, y, mask, 64, k, "bf16")
 
 
-def test_cooperative_sum_many_calls_bit_identical(full_layer):
-    """Sixty calls in a row on one stream: every call passes the grid barrier
-    (whose state carries from launch to launch) and reproduces the first
-    result bit for bit; a one-token bank shard (float32 partial y, the
-    cooperative sum writing float32) sums to the layer."""
+def test_decode_many_calls_bit_identical(full_layer):
+    """Sixty one-token calls in a row on one stream (each call's first kernel
+    starts during the previous call's last one) reproduce the first results
+    bit for bit; a one-token bank shard (float32 partial y) sums to the
+    layer."""
     wl, host, dev = full_layer
     xs = [make_tokens(wl, T=1, seed=600 + i).to(DEV) for i in range(3)]
     first = [_run_forward(dev, x, 64, 16) for x in xs]
@@ -347,7 +346,7 @@ def test_cooperative_sum_many_calls_bit_identical(full_layer):
     outs = [sfn.sparse_ffn_forward(xs[i % 3], dev["A"], dev["B"], dev["Wg"], dev["Wu"],
                                    dev["Wd"]) for i in range(60)]
     torch.cuda.synchronize()
-    assert sfn.kernel_launch_count() - c0 == 3 * 60  # h, logits + top-k, gate/up/down + sum
+    assert sfn.kernel_launch_count() - c0 == 4 * 60  # h, logits + top-k, gate/up/down, sum
     for i, (y, m) in enumerate(outs):
         assert torch.equal(y, first[i % 3][0]) and torch.equal(m, first[i % 3][1]), i
     total = torch.zeros((1, wl.d), dtype=torch.float32, device=DEV)
