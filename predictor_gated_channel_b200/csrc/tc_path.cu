@@ -34,6 +34,8 @@
 // Every mbarrier wait is bounded (async_util.cuh).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include <initializer_list>
 #include <mutex>
 #include <type_traits>
@@ -42,6 +44,39 @@
 #include "tc_util.cuh"
 
 namespace sfn {
+
+// ------------------------------------------------------------------ tensor maps
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+}  // namespace
+
+bool encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// Row-major bf16 matrix [outer][inner] with rows `stride` elements apart
+// (0: inner), box {box_inner, box_outer}, 128-byte swizzle, zero fill
+// outside.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer, uint64_t stride) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {(stride ? stride : inner) * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 namespace {
 
@@ -93,6 +128,8 @@ struct TcParams {
   bool b_once;            // the B operand (weights) is read once (one token tile): its
                           // loads carry an evict-first L2 policy
   bool accumulate;        // float32 products: add to the output instead of overwriting
+  int n_valid;            // float32 products: output columns (the last N tile may run
+                          // past them: its loads zero-fill, its stores skip them)
   unsigned *err;
 };
 
@@ -316,8 +353,13 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           if (Tr::kGateUpB) {
             load_b(b, &tB, kb * kBK, nb * (p.bn / 2), &full[s]);
             load_b(b + (p.bn / 2) * 128, &tB2, kb * kBK, nb * (p.bn / 2), &full[s]);
+          } else if (kEpi == kEpiDown) {
+            // [K][N] storage: four boxes of 64 N-elements x 64 K-rows (N 256)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              load_b(b + q * 8192, &tB, nb * kAccCols + q * 64, kb * kBK, &full[s]);
           } else if (Tr::kBMnMajor) {
-            // [K][N] storage: bn/64 boxes of 64 N-elements x 64 K-rows
+            // float32 products, [K][N] storage: bn/64 boxes of 64 x 64
             for (int q = 0; q < p.bn / 64; ++q)
               load_b(b + q * 8192, &tB, nb * p.bn + q * 64, kb * kBK, &full[s]);
           } else {
@@ -472,7 +514,7 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + c0, v);
           tmem_ld_wait();
-          if (valid && Tr::kF32) {
+          if (valid && Tr::kF32 && nb * p.bn + c0 < p.n_valid) {
             // C (=, +=) A B, float32 [M][ld_out]
             float *dst = reinterpret_cast<float *>(p.out) + t * p.ld_out + nb * p.bn + c0;
             if (p.accumulate) {
@@ -493,7 +535,7 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
                 reinterpret_cast<uint4 *>(dst)[i] =
                     make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
-          } else if (valid) {
+          } else if (valid && !Tr::kF32) {
             const int col = nb * p.bn + c0;
             if (kEpi != kEpiDown || p.ksplit > 1 || p.f32_out) {
               // fp32 logits, or fp32 partial sums [T][ksplit][ld_out]
@@ -688,36 +730,6 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-bool encoder() {
-  std::call_once(g_encode_once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void *fn = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return g_encode != nullptr;
-}
-
-// Row-major bf16 matrix [outer][inner] with rows `stride` elements apart
-// (0: inner), box {box_inner, box_outer}, 128-byte swizzle, zero fill
-// outside.
-bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-              uint32_t box_inner, uint32_t box_outer, uint64_t stride = 0) {
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {(stride ? stride : inner) * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int kEpi>
 cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtensorMap &tB2,
                       TcParams p, int num_sms, cudaStream_t st) {
@@ -990,14 +1002,17 @@ cudaError_t launch_tc_down(const FwdShape &s, const DeviceInfo &dev, const uint1
 // C[M][ldc] (=, or += when accumulate) A B: bf16 operands, float32
 // accumulation and output.  A is [M][K] (lda elements per row), or [K][M]
 // when a_mn; B is [N][K] (ldb), or [K][N] when b_mn.  N must be a multiple of
-// 64; M and K are arbitrary (the loads zero-fill past them).
+// 64; M and K are arbitrary (the loads zero-fill past them).  The N tile is
+// 256 wide from N = 256 up, with the last one cut at N (so N = 448 runs as
+// two wide tiles rather than seven 64-wide ones, which keep the MMA pipe far
+// from busy).
 cudaError_t launch_tc_gemm_f32(const DeviceInfo &dev, int M, int N, int K, const void *A,
                                int lda, bool a_mn, const void *B, int ldb, bool b_mn, float *C,
                                int ldc, bool accumulate, cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
   if (M <= 0 || K <= 0 || N <= 0 || N % 64 != 0 || (a_mn && !b_mn)) return cudaErrorInvalidValue;
   const int tiles_m = (M + kBM - 1) / kBM;
-  const int bn = pick_bn(tiles_m, N, {256, 128, 64}, dev.num_sms);
+  const int bn = N >= 256 ? 256 : N;
   CUtensorMap mA, mB;
   const bool okA = a_mn ? make_map(&mA, A, (uint64_t)M, (uint64_t)K, 64, 64, (uint64_t)lda)
                         : make_map(&mA, A, (uint64_t)K, (uint64_t)M, 64, kBM, (uint64_t)lda);
@@ -1008,13 +1023,14 @@ cudaError_t launch_tc_gemm_f32(const DeviceInfo &dev, int M, int N, int K, const
   p.T = M;
   p.err = dev.err;
   p.tiles_m = tiles_m;
-  p.tiles_n = N / bn;
+  p.tiles_n = (N + bn - 1) / bn;
   p.k_blocks = (K + kBK - 1) / kBK;
   p.ksplit = 1;
   p.bn = bn;
   p.out = C;
   p.ld_out = ldc;
   p.accumulate = accumulate;
+  p.n_valid = N;
   if (a_mn) return launch_tc<kEpiF32MM>(mA, mB, mB, p, dev.num_sms, st);
   if (b_mn) return launch_tc<kEpiF32KM>(mA, mB, mB, p, dev.num_sms, st);
   return launch_tc<kEpiF32KK>(mA, mB, mB, p, dev.num_sms, st);

@@ -155,4 +155,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Host: the driver's tensor-map encoder (false if unavailable), and a
+// row-major bf16 matrix [outer][inner] (rows `stride` elements apart, 0:
+// inner) as a 2-D map with box {box_inner, box_outer}, 128-byte swizzle and
+// zero fill outside the matrix.
+bool encoder();
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer, uint64_t stride = 0);
+
 }  // namespace sfn

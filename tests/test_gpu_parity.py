@@ -243,9 +243,10 @@ def test_zero_tokens(full_layer):
 
 # ------------------------------------------------------------------ tensor path
 
-@pytest.mark.parametrize("T", [1, 5, 64, 128, 130, 300])
+@pytest.mark.parametrize("T", [1, 5, 16, 64, 100, 128, 130, 300])
 def test_tensor_path_full_width(T, full_layer):
-    """The tcgen05 path (forced) against the oracle, every token checked."""
+    """The tcgen05 path (forced) against the oracle, every token checked: one
+    token tile (T <= 128) and several (130, 300)."""
     wl, host, dev = full_layer
     x = make_tokens(WORKLOADS["prefill"], T=T, seed=100 + T)
     y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
@@ -265,15 +266,17 @@ def test_tensor_path_k_variants(k, full_layer):
     _check_forward(host, x, y, mask, 64, k, "bf16", rows=rows)
 
 
+@pytest.mark.parametrize("T", [64, 130])
 @pytest.mark.parametrize("k", [1, 4, 16, 20, 63])
-def test_tensor_topk_exact_ties(k):
+def test_tensor_topk_exact_ties(T, k):
     """One-hot tokens and small-integer A and B make the tensor-core logits
     exact integers; every bank of B holds 16 rows four times each, so exact
     ties are everywhere.  The mask of the top-k fused into the logits GEMM
     equals the oracle's bit for bit (ties to the lower channel), for k below
-    16, at 16 and above 16 (the wider-staging variant)."""
+    16, at 16 and above 16 (the wider-staging variant), with one token tile
+    (64 tokens: the single-tile loops) and several (130)."""
     rng = np.random.default_rng(300 + k)
-    T, d, d_i, r = 130, 256, 1024, 64
+    d, d_i, r = 256, 1024, 64
     x, A, B, W, p = _tie_layer(rng, d, d_i, r, 64, T)
     _, mask = sfn.sparse_ffn_forward(_bf16_dev(x), _bf16_dev(A), _bf16_dev(B), _bf16_dev(W),
                                      _bf16_dev(W), _bf16_dev(W), bank=64, k=k, path="tensor")
