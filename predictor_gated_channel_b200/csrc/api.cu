@@ -307,12 +307,20 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
       e = timed(SFN_STAGE_TC_H, st,
                 [&] { return launch_tc_h(s, dev, x, A, h2, nullptr, 1, st); });
     }
-    if (e == cudaSuccess)
-      e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
-                [&] { return launch_tc_logits(s, dev, h2, B, nullptr, m, sig, st); });
-    if (e == cudaSuccess)
-      e = timed(SFN_STAGE_TC_GATEUP, st,
-                [&] { return launch_tc_gateup(s, dev, x, Wg, Wu, m, sig, act, st); });
+    if (tc_fused_gateup_ok(s)) {
+      // one token tile: logits, bank top-k and the masked gate/up in one kernel
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_TC_GATEUP, st, [&] {
+          return launch_tc_logits_gateup(s, dev, h2, B, x, Wg, Wu, mask, act, st);
+        });
+    } else {
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_TC_LOGITS_TOPK, st,
+                  [&] { return launch_tc_logits(s, dev, h2, B, nullptr, m, sig, st); });
+      if (e == cudaSuccess)
+        e = timed(SFN_STAGE_TC_GATEUP, st,
+                  [&] { return launch_tc_gateup(s, dev, x, Wg, Wu, m, sig, act, st); });
+    }
     if (p.ksplit > 1) {
       float *part = reinterpret_cast<float *>(w + p.off_part);
       if (e == cudaSuccess)

@@ -321,6 +321,13 @@ cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uin
 cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
                              const void *Wg, const void *Wu, const uint64_t *mask,
                              const float *sig, uint16_t *act, cudaStream_t st);
+// With all tokens in one 128-row tile: the logits GEMM, the bank top-k and
+// the masked gate/up in one kernel (mask may be null).
+bool tc_fused_gateup_ok(const FwdShape &s);
+cudaError_t launch_tc_logits_gateup(const FwdShape &s, const DeviceInfo &dev,
+                                    const uint16_t *h2, const void *B, const void *x,
+                                    const void *Wg, const void *Wu, uint64_t *mask,
+                                    uint16_t *act, cudaStream_t st);
 cudaError_t launch_tc_dense4x_gateup(const FwdShape &s, const DeviceInfo &dev, const void *x,
                                      const void *Wg, const void *Wu, uint64_t *mask,
                                      uint16_t *act, cudaStream_t st);

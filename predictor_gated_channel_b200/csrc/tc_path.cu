@@ -729,6 +729,274 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------- one token tile: G2 + G3
+// With all tokens in one tile, the logits GEMM (G2) is folded into the
+// gate/up GEMM (G3): a unit is 128 channels (two banks), and its K sequence
+// is first the r/64 logits blocks (A = H hi and H lo, B = the banks' rows of
+// B), then the d/64 gate/up blocks (A = x, B = the channels' W_gate and
+// W_up rows).  The logits accumulator (TMEM columns [256, 384)) completes
+// early; the epilogue ranks the two banks from it while the MMA warp goes on
+// with the gate/up blocks, and keeps each row's mask word and the kept
+// channels' sigma for the gate/up epilogue of the same (row, bank) -- the same
+// thread, so nothing crosses warps.  The separate logits kernel, its ramp and
+// its top-k tail disappear; the top-k work overlaps the weight stream.
+struct G23Params {
+  int64_t T;
+  int n_units;            // d_i / 128
+  int kb_l, kb_gu;        // logits blocks (r / 64), gate/up blocks (d / 64)
+  int stages;
+  uint32_t stage_bytes, a_tile_bytes, tx_l, tx_gu;
+  uint32_t idesc_l, idesc_gu;
+  int r, k, n_banks, ld_out;
+  uint16_t *act;          // [T][d_i] bf16
+  uint64_t *mask;         // [T][n_banks], or null
+  unsigned *err;
+};
+
+constexpr int kG23EpiWarps = 8;
+constexpr int kG23Threads = (2 + kG23EpiWarps) * 32;
+
+__global__ void __launch_bounds__(kG23Threads, 1)
+    k_tc_logits_gateup(const __grid_constant__ CUtensorMap tH,
+                       const __grid_constant__ CUtensorMap tBw,
+                       const __grid_constant__ CUtensorMap tX,
+                       const __grid_constant__ CUtensorMap tG,
+                       const __grid_constant__ CUtensorMap tU, const G23Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)p.stages * p.stage_bytes);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + p.stages;
+  uint64_t *lfull = bars + 2 * p.stages, *lempty = lfull + 1;
+  uint64_t *gfull = lfull + 2, *gempty = lfull + 3;
+  uint64_t *done = lfull + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  float *stage_rows = reinterpret_cast<float *>(smem + (size_t)p.stages * p.stage_bytes + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nblk = p.kb_l + p.kb_gu;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(lfull, 1);
+    mbar_init(lempty, kG23EpiWarps * 32);
+    mbar_init(gfull, 1);
+    mbar_init(gempty, kG23EpiWarps * 32);
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * kAccCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  if (warp != 0) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tH);
+      prefetch_tmap(&tBw);
+      prefetch_tmap(&tX);
+      prefetch_tmap(&tG);
+      prefetch_tmap(&tU);
+      // every weight byte is read once: evict-first
+      const uint64_t once = make_evict_first_policy();
+      auto issue_w = [&](int s, int i, int nb) {  // weights of block i
+        unsigned char *st = smem + (size_t)s * p.stage_bytes;
+        if (i < p.kb_l) {
+          tma_load_2d_hint(st + 2 * p.a_tile_bytes, &tBw, i * kBK, nb * 128, &full[s], once);
+        } else {
+          const int kb = i - p.kb_l;
+          tma_load_2d_hint(st + p.a_tile_bytes, &tG, kb * kBK, nb * 128, &full[s], once);
+          tma_load_2d_hint(st + p.a_tile_bytes + 16384, &tU, kb * kBK, nb * 128, &full[s], once);
+        }
+      };
+      auto issue_t = [&](int s, int i) {  // token operand of block i
+        unsigned char *st = smem + (size_t)s * p.stage_bytes;
+        if (i < p.kb_l) {
+          tma_load_2d(st, &tH, i * kBK, 0, &full[s]);
+          tma_load_2d(st + p.a_tile_bytes, &tH, p.r + i * kBK, 0, &full[s]);
+        } else {
+          tma_load_2d(st, &tX, (i - p.kb_l) * kBK, 0, &full[s]);
+        }
+      };
+      // before the dependency wait: the first unit's first stages' weights
+      int pre = 0;
+      if ((int)blockIdx.x < p.n_units) {
+        pre = min(p.stages, nblk);
+        for (int j = 0; j < pre; ++j) {
+          mbar_arrive_expect_tx(&full[j], j < p.kb_l ? p.tx_l : p.tx_gu);
+          issue_w(j, j, blockIdx.x);
+        }
+      }
+      pdl_wait();
+      pdl_launch_dependents();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x) {
+        for (int i = 0; i < nblk; ++i, ++it) {
+          const int s = (int)(it % p.stages);
+          const uint32_t use = it / p.stages;
+          if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          if ((int)it >= pre) {
+            mbar_arrive_expect_tx(&full[s], i < p.kb_l ? p.tx_l : p.tx_gu);
+            issue_w(s, i, unit);
+          }
+          issue_t(s, i);
+        }
+      }
+      const uint32_t issued = it > (uint32_t)pre ? it : (uint32_t)pre;
+      for (int s = 0; s < p.stages && (uint32_t)s < issued; ++s) {
+        const uint32_t last = s + ((issued - 1 - s) / p.stages) * p.stages;
+        mbar_wait(&full[s], (last / p.stages) & 1u, p.err);
+      }
+    } else {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t d_gu = tmem_base, d_l = tmem_base + kAccCols;
+      uint32_t it = 0, lt = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++lt) {
+        for (int i = 0; i < nblk; ++i, ++it) {
+          // single accumulators: before a unit's first logits (gate/up) MMA,
+          // the previous unit's epilogue must have read them
+          if (lt > 0 && i == 0 && !mbar_wait(lempty, (lt - 1) & 1u, p.err)) ok = false;
+          if (lt > 0 && i == p.kb_l && !mbar_wait(gempty, (lt - 1) & 1u, p.err)) ok = false;
+          if (!ok) break;
+          const int s = (int)(it % p.stages);
+          if (!mbar_wait(&full[s], (it / p.stages) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const unsigned char *st = smem + (size_t)s * p.stage_bytes;
+          if (i < p.kb_l) {
+            const uint64_t ah = desc_kmajor_sw128(st);
+            const uint64_t al = desc_kmajor_sw128(st + p.a_tile_bytes);
+            const uint64_t bd = desc_kmajor_sw128(st + 2 * p.a_tile_bytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              umma_f16(d_l, ah + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), p.idesc_l,
+                       (i > 0 || kk > 0) ? 1u : 0u);
+              umma_f16(d_l, al + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), p.idesc_l, 1u);
+            }
+          } else {
+            const uint64_t ad = desc_kmajor_sw128(st);
+            const uint64_t bd = desc_kmajor_sw128(st + p.a_tile_bytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              umma_f16(d_gu, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), p.idesc_gu,
+                       (i > p.kb_l || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          if (i == p.kb_l - 1) umma_commit(lfull);
+          if (i == nblk - 1) umma_commit(gfull);
+        }
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;           // token row of the tile
+    const int h = (warp - 2) >> 2;           // this thread's bank of the unit
+    const int64_t t = row;
+    const bool valid = t < p.T;
+    const int srow = p.k | 1;
+    float *stg = stage_rows + (h * kBM + row) * srow;
+    uint32_t lt = 0;
+    for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++lt) {
+      const int bank = unit * 2 + h;
+      // 1. logits of bank h: mask word, kept channels' sigma (in stg)
+      if (!mbar_wait(lfull, lt & 1u, p.err)) break;
+      tc_fence_after();
+      const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + kAccCols + h * 64;
+      uint32_t tau;
+      int gt;
+      bank_threshold(tl, p.k, tau, gt);
+      const int need = p.k - gt;
+      int eq = 0, cnt = 0;
+      uint64_t word = 0ull;
+#pragma unroll 1
+      for (int g = 0; g < 4; ++g) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tl + g * 16, v);
+        tmem_ld_wait();
+        uint32_t b = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t key = order_key(__uint_as_float(v[i]));
+          const bool take = (key > tau) | ((key == tau) & (eq < need));
+          eq += (key == tau);
+          b |= (uint32_t)take << i;
+          if (take) stg[cnt] = __uint_as_float(v[i]);
+          cnt += take;
+        }
+        word |= (uint64_t)b << (g * 16);
+      }
+      tc_fence_before();
+      mbar_arrive(lempty);
+      for (int s1 = 0; s1 < p.k; ++s1) stg[s1] = sigmoid_fast(stg[s1]);
+      if (valid && p.mask != nullptr) p.mask[t * p.n_banks + bank] = word;
+      // 2. a = sigma(p) g u for bank h: g at columns [h*64, h*64 + 64), u at
+      //    [128 + h*64, ...) of the gate/up accumulator
+      if (!mbar_wait(gfull, lt & 1u, p.err)) break;
+      tc_fence_after();
+      const uint32_t tg = tmem_base + ((uint32_t)(q * 32) << 16);
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t g[32], u[32];
+        tmem_ld_32x32b_x32(tg + h * 64 + c0, g);
+        tmem_ld_32x32b_x32(tg + 128 + h * 64 + c0, u);
+        tmem_ld_wait();
+        if (valid) {
+          uint32_t packed[16];
+          int rank = __popcll(word & ((1ull << c0) - 1ull));
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float a2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const bool on = (word >> (c0 + i + e)) & 1ull;
+              const float sg = on ? stg[rank] : 0.f;
+              a2[e] = on ? sg * __uint_as_float(g[i + e]) * __uint_as_float(u[i + e]) : 0.f;
+              rank += on;
+            }
+            packed[i / 2] = pack_bf16x2(a2[0], a2[1]);
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(p.act + t * p.ld_out + bank * 64 + c0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
+                                packed[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(gempty);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kAccCols);
+  }
+}
+
 // ------------------------------------------------------------------ host
 template <int kEpi>
 cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const CUtensorMap &tB2,
@@ -954,6 +1222,59 @@ cudaError_t launch_tc_gateup(const FwdShape &s, const DeviceInfo &dev, const voi
   p.mask = const_cast<uint64_t *>(mask);
   p.sig = const_cast<float *>(sig);
   return launch_tc<kEpiGateUp>(mX, mG, mU, p, dev.num_sms, st);
+}
+
+// G2 + G3 at one token tile (T <= 128): logits, bank top-k and a = sigma(p) g u
+// in one kernel (k_tc_logits_gateup).  mask (may be null) receives the mask.
+bool tc_fused_gateup_ok(const FwdShape &s) {
+  return tc_shape_ok(s) && s.T <= kBM && s.d_i % 128 == 0 && s.k < 64;
+}
+
+cudaError_t launch_tc_logits_gateup(const FwdShape &s, const DeviceInfo &dev,
+                                    const uint16_t *h2, const void *B, const void *x,
+                                    const void *Wg, const void *Wu, uint64_t *mask,
+                                    uint16_t *act, cudaStream_t st) {
+  if (!encoder()) return cudaErrorNotSupported;
+  if (!tc_fused_gateup_ok(s)) return cudaErrorInvalidValue;
+  const int a_rows = a_box_rows(s);
+  CUtensorMap mH, mB, mX, mG, mU;
+  if (!make_map(&mH, h2, 2 * s.r, s.T, 64, a_rows) || !make_map(&mB, B, s.r, s.d_i, 64, 128) ||
+      !make_map(&mX, x, s.d, s.T, 64, a_rows) || !make_map(&mG, Wg, s.d, s.d_i, 64, 128) ||
+      !make_map(&mU, Wu, s.d, s.d_i, 64, 128))
+    return cudaErrorInvalidValue;
+  G23Params p{};
+  p.T = s.T;
+  p.n_units = s.d_i / 128;
+  p.kb_l = s.r / kBK;
+  p.kb_gu = s.d / kBK;
+  p.r = s.r;
+  p.k = s.k;
+  p.n_banks = s.n_banks;
+  p.ld_out = s.d_i;
+  p.act = act;
+  p.mask = mask;
+  p.err = dev.err;
+  p.a_tile_bytes = (uint32_t)a_rows * kBK * 2;
+  p.tx_l = 2 * p.a_tile_bytes + 16384;
+  p.tx_gu = p.a_tile_bytes + 32768;
+  // one stage holds either block kind; the MMA reads 128 rows from each A
+  // tile start, which stays inside the stage (a tile <= 16 KB)
+  p.stage_bytes = p.a_tile_bytes + 32768;
+  p.idesc_l = idesc_bf16_f32(kBM, 128, false);
+  p.idesc_gu = idesc_bf16_f32(kBM, 256, false);
+  const size_t epi = (size_t)2 * kBM * (s.k | 1) * sizeof(float);
+  const size_t fixed = 1024 + 256 + epi;
+  p.stages = (int)(((size_t)kMaxDynSmem - fixed) / p.stage_bytes);
+  if (p.stages > 8) p.stages = 8;
+  if (p.stages < 2 || (2 * p.stages + 5) * 8 + 4 > 256) return cudaErrorInvalidValue;
+  const size_t smem = fixed + (size_t)p.stages * p.stage_bytes;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(k_tc_logits_gateup), smem);
+  if (e != cudaSuccess) return e;
+  const int grid = p.n_units < dev.num_sms ? p.n_units : dev.num_sms;
+  e = launch_pdl(k_tc_logits_gateup, dim3(grid), dim3(kG23Threads), smem, st, mH, mB, mX, mG,
+                 mU, p);
+  count_launches(1);
+  return e;
 }
 
 // Dense-4x comparison, first GEMM: [G | U] = X [Wg; Wu]^T -> act =

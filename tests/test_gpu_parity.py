@@ -225,9 +225,10 @@ def test_outputs_do_not_spill(full_layer):
 def test_launch_counter_counts_kernels(full_layer):
     """Few tokens: h, logits + top-k, gate/up/down, the sum of the partial
     rows; many: the tensor path (h, its split-K sum, logits + top-k,
-    gate/up, down, its split-K sum at 64 tokens)."""
+    gate/up, down, its split-K sum at 64 tokens -- with one token tile the
+    logits and gate/up are one kernel)."""
     wl, host, dev = full_layer
-    for T, n in ((1, 4), (2, 4), (64, 6)):
+    for T, n in ((1, 4), (2, 4), (64, 5), (300, 6)):
         x = make_tokens(wl, T=T).to(DEV)
         c0 = sfn.kernel_launch_count()
         _run_forward(dev, x, 64, 16)
