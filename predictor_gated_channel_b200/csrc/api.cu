@@ -293,28 +293,21 @@ sfn_status forward_impl(const void *x, const void *A, const void *B, const void 
     float *sig = reinterpret_cast<float *>(w + p.off_sig);
     uint16_t *act = reinterpret_cast<uint16_t *>(w + p.off_act);
     uint64_t *m = mask ? mask : reinterpret_cast<uint64_t *>(w + p.off_mask);
-    // one token tile: logits and gate/up run as one kernel, whose first
-    // weight bytes the h GEMM brings into L2 meanwhile
-    const bool fused = tc_fused_gateup_ok(s);
-    const void *pf_g = fused ? Wg : nullptr, *pf_u = fused ? Wu : nullptr;
-    const void *pf_b = fused ? B : nullptr;
     if (p.hsplit > 1) {
       // few 128-token tiles: split K, then sum the fp32 partials and split
       // the sum into the bf16 hi/lo operand of the logits GEMM
       float *hpart = reinterpret_cast<float *>(w + p.off_hpart);
-      e = timed(SFN_STAGE_TC_H, st, [&] {
-        return launch_tc_h(s, dev, x, A, h2, hpart, p.hsplit, st, pf_g, pf_u, pf_b);
-      });
+      e = timed(SFN_STAGE_TC_H, st,
+                [&] { return launch_tc_h(s, dev, x, A, h2, hpart, p.hsplit, st); });
       if (e == cudaSuccess)
         e = timed(SFN_STAGE_REDUCE, st, [&] {
           return launch_reduce_partials(s, p.hsplit, hpart, h2, st, ReduceOut::kSplitH);
         });
     } else {
-      e = timed(SFN_STAGE_TC_H, st, [&] {
-        return launch_tc_h(s, dev, x, A, h2, nullptr, 1, st, pf_g, pf_u, pf_b);
-      });
+      e = timed(SFN_STAGE_TC_H, st,
+                [&] { return launch_tc_h(s, dev, x, A, h2, nullptr, 1, st); });
     }
-    if (fused) {
+    if (tc_fused_gateup_ok(s)) {
       // one token tile: logits, bank top-k and the masked gate/up in one kernel
       if (e == cudaSuccess)
         e = timed(SFN_STAGE_TC_GATEUP, st, [&] {

@@ -313,12 +313,8 @@ int tc_down_splits(const FwdShape &s, int num_sms);
 int tc_h_splits(const FwdShape &s, int num_sms);
 bool tc_shape_ok(const FwdShape &s);
 TcPlan plan_tc(const FwdShape &s);
-// pf_g, pf_u, pf_b (all or none): weights of the fused logits + gate/up
-// kernel that runs next, whose first bytes this GEMM prefetches into L2.
 cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
-                        uint16_t *h2, float *partial, int ksplit, cudaStream_t st,
-                        const void *pf_g = nullptr, const void *pf_u = nullptr,
-                        const void *pf_b = nullptr);
+                        uint16_t *h2, float *partial, int ksplit, cudaStream_t st);
 cudaError_t launch_tc_logits(const FwdShape &s, const DeviceInfo &dev, const uint16_t *h2,
                              const void *B, float *logits, uint64_t *mask, float *sig,
                              cudaStream_t st);

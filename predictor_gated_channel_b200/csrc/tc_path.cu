@@ -87,10 +87,6 @@ constexpr uint32_t kTileA = kBM * kBK * 2;     // 16 KB
 constexpr int kAccCols = 256;                  // TMEM columns per accumulator
 constexpr size_t kMaxDynSmem = 232448;            // 227 KB per CTA on sm_100
 constexpr int kGroupM = 8;                     // tile rasterisation group
-// One token tile: K blocks of each W_gate / W_up row that the h GEMM brings
-// into L2 for the fused logits + gate/up kernel (2 KB of each 8 KB row at
-// d = 4096: 59 MB, about as much as DRAM serves while h and its split-K sum run)
-constexpr int kPrefetchBlocks = 16;
 
 enum : int {
   kEpiHSplit = 0,
@@ -134,14 +130,6 @@ struct TcParams {
   bool accumulate;        // float32 products: add to the output instead of overwriting
   int n_valid;            // float32 products: output columns (the last N tile may run
                           // past them: its loads zero-fill, its stores skip them)
-  // h GEMM only, optional: weights the next kernel reads, brought into L2 while
-  // this small GEMM leaves DRAM mostly idle -- the first pf_row_bytes of each of
-  // the pf_rows rows (pf_row_stride bytes apart) of pf_rows0 and pf_rows1, and
-  // all pf_block_bytes of pf_block
-  const char *pf_rows0, *pf_rows1, *pf_block;
-  uint32_t pf_row_bytes;
-  int pf_rows;
-  int64_t pf_row_stride, pf_block_bytes;
   unsigned *err;
 };
 
@@ -483,22 +471,6 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
     const int q = warp & 3;           // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;    // token row inside the tile
     const int half_id = (warp - 2) >> 2;  // which of a quadrant's epilogue warps
-    if (kEpi == kEpiHSplit && p.pf_rows0 != nullptr) {
-      // after the dependency wait (the previous call's streams are done): the
-      // next kernel's first weight bytes into L2, spread over the grid's
-      // epilogue threads
-      const int et = threadIdx.x - 64;
-      const int64_t gt = (int64_t)blockIdx.x * (Tr::kEpiWarps * 32) + et;
-      const int64_t nt = (int64_t)gridDim.x * (Tr::kEpiWarps * 32);
-      for (int64_t rr = gt; rr < p.pf_rows; rr += nt) {
-        prefetch_l2(p.pf_rows0 + rr * p.pf_row_stride, p.pf_row_bytes);
-        prefetch_l2(p.pf_rows1 + rr * p.pf_row_stride, p.pf_row_bytes);
-      }
-      for (int64_t o = gt * 16384; o < p.pf_block_bytes; o += nt * 16384) {
-        const int64_t rest = p.pf_block_bytes - o;
-        prefetch_l2(p.pf_block + o, (uint32_t)(rest < 16384 ? rest : 16384));
-      }
-    }
     uint32_t lt = 0;
     for (int unit = blockIdx.x; unit < total; unit += gridDim.x, ++lt) {
       int mb, nb, kb0, kb1;
@@ -1150,8 +1122,7 @@ int tc_h_splits(const FwdShape &s, int num_sms) {
 // ksplit > 1: fp32 partial sums [T][ksplit][r] into `partial` (the caller
 // reduces them and splits hi/lo).
 cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x, const void *A,
-                        uint16_t *h2, float *partial, int ksplit, cudaStream_t st,
-                        const void *pf_g, const void *pf_u, const void *pf_b) {
+                        uint16_t *h2, float *partial, int ksplit, cudaStream_t st) {
   if (!encoder()) return cudaErrorNotSupported;
   const int tiles_m = (int)((s.T + kBM - 1) / kBM);
   const int bn_h = ksplit > 1 ? 64
@@ -1164,17 +1135,6 @@ cudaError_t launch_tc_h(const FwdShape &s, const DeviceInfo &dev, const void *x,
   p.k_blocks = s.d / kBK;
   p.ksplit = ksplit;
   p.bn = bn_h;
-  if (pf_g != nullptr && pf_u != nullptr && pf_b != nullptr) {
-    // the fused logits + gate/up kernel's first blocks: all of B, and the
-    // first kPrefetchBlocks K blocks of every W_gate and W_up row
-    p.pf_rows0 = static_cast<const char *>(pf_g);
-    p.pf_rows1 = static_cast<const char *>(pf_u);
-    p.pf_block = static_cast<const char *>(pf_b);
-    p.pf_rows = s.d_i;
-    p.pf_row_stride = (int64_t)s.d * 2;
-    p.pf_row_bytes = (uint32_t)std::min<int64_t>((int64_t)s.d * 2, kPrefetchBlocks * kBK * 2);
-    p.pf_block_bytes = (int64_t)s.d_i * s.r * 2;
-  }
   if (ksplit > 1) {
     p.out = partial;
     p.ld_out = s.r;
