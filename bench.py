@@ -313,7 +313,8 @@ def extra_workloads_wanted(args, world):
 def summarize(line):
     """The per-workload entry of the headline line."""
     keys = ("value", "unit", "steps", "warmup", "ms_per_step", "roofline", "step_roofline",
-            "mask_union_channels", "clocks", "gpu_launches", "step_time_spread", "e2e")
+            "mask_union_channels", "clocks", "gpu_launches", "step_time_spread", "e2e",
+            "cpu_baseline")
     out = {k: line.get(k) for k in keys}
     out["workload"] = line["config"]["workload"]
     out["dtype"] = line["dtype"]
@@ -540,6 +541,10 @@ def measure(args, workload, K, W, rank, world, dev, L, main):
     for v in stages.values():
         v["share"] = v["ms_total"] / tot
     work = stage_work(wl, T, union)
+    if "tc_gateup" in stages and "tc_logits_topk" not in stages:
+        # one token tile: the logits GEMM and its top-k run inside the gate/up kernel
+        work["tc_gateup"] = {k: work["tc_gateup"][k] + work["tc_logits_topk"][k]
+                             for k in ("bytes", "flops")}
     bound = "hbm" if T <= 256 else "tensor"
     if "tc_down" in stages and "reduce" in stages:  # split-K partial sums
         work["reduce"] = {"bytes": T * wl.d * 4, "flops": 0}
@@ -599,9 +604,10 @@ def measure(args, workload, K, W, rank, world, dev, L, main):
                "steps": n_e2e}
 
     cpu = None
-    if main and rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the workloads beside the headline line take a shorter sample
         cpu = cpu_baseline(wl, {k: v.cpu() for k, v in layers[0].items()}, xs[0].cpu(),
-                           method=args.method)
+                           budget_s=15.0 if main else 5.0, method=args.method)
 
     if world > 1:
         dist.barrier()
