@@ -580,17 +580,28 @@ def measure(args, workload, K, W, rank, world, dev, L, main):
             e0.record(stream)
             for j in range(n_e2e):
                 i = j % S
+                # host input in, the C ABI call, host output back: what a caller does
                 x_dev.copy_(x_host[i], non_blocking=True)
                 lay = layers[i]
                 if dense4x:
-                    sfn.dense4x_forward(x_dev, lay["Wg"], lay["Wu"], lay["Wd"], bank=wl.bank,
-                                        k=wl.k, y=ys[i], mask=ms[i], workspace=ws,
-                                        stream=stream)
+                    rc = L.sfn_dense4x_forward(x_dev.data_ptr(), lay["Wg"].data_ptr(),
+                                               lay["Wu"].data_ptr(), lay["Wd"].data_ptr(),
+                                               ys[i].data_ptr(), ms[i].data_ptr(), T, wl.d,
+                                               wl.d_i, wl.bank, wl.k, ws.data_ptr(), ws_bytes,
+                                               stream.cuda_stream)
+                elif wl.dtype == "bf16":
+                    rc = L.sfn_sparse_ffn_forward_path(
+                        x_dev.data_ptr(), lay["A"].data_ptr(), lay["B"].data_ptr(),
+                        lay["Wg"].data_ptr(), lay["Wu"].data_ptr(), lay["Wd"].data_ptr(),
+                        ys[i].data_ptr(), ms[i].data_ptr(), T, wl.d, wl.d_i, wl.r, wl.bank,
+                        wl.k, path_id, ws.data_ptr(), ws_bytes, stream.cuda_stream)
                 else:
-                    sfn.sparse_ffn_forward(x_dev, lay["A"], lay["B"], lay["Wg"], lay["Wu"],
-                                           lay["Wd"], bank=wl.bank, k=wl.k, y=ys[i],
-                                           mask=ms[i], workspace=ws, path=args.path,
-                                           stream=stream)
+                    rc = L.sfn_sparse_ffn_forward_f32_ws(
+                        x_dev.data_ptr(), lay["A"].data_ptr(), lay["B"].data_ptr(),
+                        lay["Wg"].data_ptr(), lay["Wu"].data_ptr(), lay["Wd"].data_ptr(),
+                        ys[i].data_ptr(), ms[i].data_ptr(), T, wl.d, wl.d_i, wl.r, wl.bank,
+                        wl.k, ws.data_ptr(), ws_bytes, stream.cuda_stream)
+                _capi.check(rc, "e2e forward")
                 y_host.copy_(ys[i], non_blocking=True)
                 m_host.copy_(ms[i], non_blocking=True)
                 stream.synchronize()  # the caller reads the step's result
