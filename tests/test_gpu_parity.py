@@ -256,14 +256,17 @@ def test_tensor_path_full_width(T, full_layer):
     _check_forward(host, x, y, mask, 64, 16, "bf16")
 
 
+@pytest.mark.parametrize("T", [100, 160])
 @pytest.mark.parametrize("k", [1, 16, 63, 64])
-def test_tensor_path_k_variants(k, full_layer):
+def test_tensor_path_k_variants(T, k, full_layer):
+    """k below, at and above 16 and k = bank on the tensor path, with one
+    token tile (100 tokens: the fused logits + gate/up kernel) and two."""
     wl, host, dev = full_layer
-    x = make_tokens(WORKLOADS["prefill"], T=160, seed=200 + k)
+    x = make_tokens(WORKLOADS["prefill"], T=T, seed=200 + k)
     y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
                                      dev["Wd"], k=k, path="tensor")
     torch.cuda.synchronize()
-    rows = np.arange(0, 160, 7)
+    rows = np.arange(0, T, 7)
     _check_forward(host, x, y, mask, 64, k, "bf16", rows=rows)
 
 
