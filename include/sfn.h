@@ -211,7 +211,9 @@ sfn_status sfn_sparse_ffn_forward_static(const void *x, const void *A, const voi
  *   SFN_PATH_TENSOR     tcgen05 tensor-core GEMMs over 128-token tiles with
  *                       the top-k and the sigma(p) g u mask fused into their
  *                       epilogues (bf16, bank 64, d and d_i multiples of
- *                       256, r a multiple of 64 up to 512);
+ *                       256, r a multiple of 64 up to 512); when all tokens
+ *                       fit one tile (T <= 128) the logits GEMM, the top-k
+ *                       and the masked gate/up are one kernel;
  *   SFN_PATH_AUTO       the tensor path from T >= 6 when the shape allows
  *                       it, the CUDA-core path otherwise.
  */
