@@ -369,6 +369,22 @@ def test_decode_many_calls_bit_identical(full_layer):
     assert (total - ref).abs().max().item() <= 2e-2 * ref.abs().max().item()
 
 
+def test_one_tile_kernel_several_units_per_cta():
+    """With more 128-channel units than SMs (here 304), each CTA of the fused
+    one-tile logits + gate/up kernel takes several units in turn, reusing its
+    single logits and gate/up accumulators; every token checked."""
+    import math
+    from predictor_gated_channel_b200.inputs import Workload
+    wl = Workload("wide", 64, 256, 38912, 64, 64, 16, "bf16", "rmsnorm", 1.0 / math.sqrt(9728))
+    host = make_layer(wl, seed=9)
+    dev = {n: v.to(DEV) for n, v in host.items()}
+    x = make_tokens(wl, seed=9)
+    y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
+                                     dev["Wd"], path="tensor")
+    torch.cuda.synchronize()
+    _check_forward(host, x, y, mask, wl.bank, wl.k, "bf16")
+
+
 def test_paths_agree(full_layer):
     """CUDA-core and tensor paths on the same 96 tokens: masks differ only at
     allowed near-ties, outputs within the bf16 tolerance of each other."""
