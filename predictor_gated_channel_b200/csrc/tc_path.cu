@@ -159,14 +159,16 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
   nb = idx / gm;
 }
 
-// Work unit -> output tile and its K-block range [kb0, kb1).
+// Work unit -> output tile and its K-block range [kb0, kb1).  The K splits
+// differ in length by at most one block, so none is empty while ksplit <=
+// k_blocks (equal ceil-sized ranges would leave the last splits empty when
+// ksplit does not divide k_blocks).
 __device__ __forceinline__ void unit_coords(int unit, const TcParams &p, int &mb, int &nb,
                                             int &kb0, int &kb1) {
   const int split = unit % p.ksplit;
   tile_coords(unit / p.ksplit, p.tiles_m, p.tiles_n, mb, nb);
-  const int per = (p.k_blocks + p.ksplit - 1) / p.ksplit;
-  kb0 = split * per;
-  kb1 = min(p.k_blocks, kb0 + per);
+  kb0 = (int)((int64_t)p.k_blocks * split / p.ksplit);
+  kb1 = (int)((int64_t)p.k_blocks * (split + 1) / p.ksplit);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__(EpiTraits<kEpi>::kThreads, 1)
           if ((int)blockIdx.x < total) {
             int mb, nb, kb0, kb1;
             unit_coords(blockIdx.x, p, mb, nb, kb0, kb1);
-            pre = min(p.stages, kb1 - kb0);
+            pre = max(0, min(p.stages, kb1 - kb0));
             for (int j = 0; j < pre; ++j) {
               mbar_arrive_expect_tx(&full[j], p.tx_bytes);
               issue_b(j, kb0 + j, nb);
