@@ -14,7 +14,7 @@ import parity
 import predictor_gated_channel_b200 as sfn
 from predictor_gated_channel_b200 import _capi
 from predictor_gated_channel_b200 import build as sfn_build
-from predictor_gated_channel_b200.inputs import WORKLOADS, make_layer, make_tokens
+from predictor_gated_channel_b200.inputs import WORKLOADS, Workload, make_layer, make_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -379,6 +379,23 @@ def test_one_tile_kernel_several_units_per_cta():
     host = make_layer(wl, seed=9)
     dev = {n: v.to(DEV) for n, v in host.items()}
     x = make_tokens(wl, seed=9)
+    y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
+                                     dev["Wd"], path="tensor")
+    torch.cuda.synchronize()
+    _check_forward(host, x, y, mask, wl.bank, wl.k, "bf16")
+
+
+@pytest.mark.parametrize("T", [64, 200])
+def test_tensor_path_uneven_k_splits(T):
+    """Split-K counts that do not divide the K-block count: d = 1280 gives the
+    h GEMM 20 K blocks over 8 splits at one token tile, d_i = 2816 the down
+    GEMM 44 over 8.  Each split must get a non-empty range; every token is
+    checked."""
+    wl = Workload("uneven", T, 1280, 2816, 64, 64, 16, "bf16", "rmsnorm",
+                  1.0 / math.sqrt(704))
+    host = make_layer(wl, seed=13)
+    dev = {n: v.to(DEV) for n, v in host.items()}
+    x = make_tokens(wl, seed=13)
     y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
                                      dev["Wd"], path="tensor")
     torch.cuda.synchronize()
