@@ -23,8 +23,8 @@
  * notes of the repository):
  *   - predictor is a plain linear factorisation p = B (A x), no bias, no
  *     inner activation;
- *   - the predictor "replaces the dense SwiGLU gate sigma(u)": silu(g) =
- *     g*sigma(g) becomes g*sigma(p), so a_j = sigma(p_j) * g_j * u_j with
+ *   - the predictor's logits take the place of the dense SwiGLU gate's
+ *     sigma: silu(g) = g*sigma(g) becomes g*sigma(p), so a_j = sigma(p_j) * g_j * u_j with
  *     g_j = Wg[j].x and u_j = Wu[j].x;
  *   - banks are contiguous index ranges [b*bank, (b+1)*bank);
  *   - ranking is on p (not sigma(p)); equal logits go to the lower index;
@@ -64,7 +64,7 @@ double sfn_oracle_sigmoid(double z) {
   return e / (1.0 + e);
 }
 
-/* Predictor, "R^d -> R^448 -> R^{d_i}":  h = A x  (A is [r][d]),  p = B h
+/* Predictor, a two-layer map R^d -> R^448 -> R^{d_i}:  h = A x  (A is [r][d]),  p = B h
  * (B is [d_i][r]).  logits is [T][d_i] double. */
 void sfn_oracle_predict(const void *x, int x_dt, const void *A, int A_dt,
                         const void *B, int B_dt, int64_t T, int d, int d_i,
@@ -165,7 +165,7 @@ void sfn_oracle_forward(const void *x, int x_dt, const void *A, int A_dt,
                                 Wu_dt, Wd, Wd_dt, T, d, d_i, bank, y);
 }
 
-/* The pages' own "functional simulation" form: materialise the dense gate
+/* The form of the pages' own GPU code, which simulates the sparsity: materialise the dense gate
  * and up projections for every channel, form the predictor-gated product,
  * multiply by the 0/1 mask, then run the dense down projection.  A separate
  * loop nest from sfn_oracle_forward_given_mask, used to check that skipping

@@ -1,8 +1,8 @@
 // gather_ffn.cu -- sparse gate/up/down over the kept channels only, on CUDA
 // cores (the few-token path).
 //
-// "Inactive channels are exactly zero" and the gate, up and down projections
-// skip them: "Continual LLM Upcycling: A Predictor-Gated Bank-Wise Sparsity
+// Channels outside the mask are exactly zero in the forward pass, so the gate,
+// up and down projections may skip them: "Continual LLM Upcycling: A Predictor-Gated Bank-Wise Sparsity
 // Training Recipe for Dense-to-Sparse LLMs", gist.science summary,
 // "1. Architectuur" (Executie / Forward Pass) and "3. Hardware Implicaties".
 //

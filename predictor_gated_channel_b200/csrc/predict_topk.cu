@@ -1,7 +1,8 @@
 // predict_topk.cu -- CUDA-core kernels of the predictor and the bank top-k
 // (the few-token path, and the standalone top-k).
 //
-// Predictor "R^d -> R^448 -> R^{d_i}" and the bank-wise hard top-16 of 64:
+// The predictor, a two-layer map R^d -> R^448 -> R^{d_i}, and the bank-wise
+// hard top-16 of 64:
 // "Continual LLM Upcycling: A Predictor-Gated Bank-Wise Sparsity Training
 // Recipe for Dense-to-Sparse LLMs", gist.science summary, "1. Architectuur".
 //
