@@ -128,7 +128,7 @@ def test_forward_tiny_f32():
     assert n_diff == 0
 
 
-@pytest.mark.parametrize("T", [1, 3, 17, 64])
+@pytest.mark.parametrize("T", [1, 3, 5, 6, 17, 64])
 def test_forward_full_width_bf16(T, full_layer):
     wl, host, dev = full_layer
     x = make_tokens(wl, T=T, seed=T)
@@ -244,10 +244,11 @@ def test_zero_tokens(full_layer):
 
 # ------------------------------------------------------------------ tensor path
 
-@pytest.mark.parametrize("T", [1, 5, 16, 64, 100, 128, 130, 300])
+@pytest.mark.parametrize("T", [1, 5, 6, 16, 64, 100, 127, 128, 129, 130, 256, 257, 300])
 def test_tensor_path_full_width(T, full_layer):
     """The tcgen05 path (forced) against the oracle, every token checked: one
-    token tile (T <= 128) and several (130, 300)."""
+    token tile (T <= 128) and several, with full and ragged last tiles on
+    both sides of the tile boundaries."""
     wl, host, dev = full_layer
     x = make_tokens(WORKLOADS["prefill"], T=T, seed=100 + T)
     y, mask = sfn.sparse_ffn_forward(x.to(DEV), dev["A"], dev["B"], dev["Wg"], dev["Wu"],
