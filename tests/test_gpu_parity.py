@@ -202,6 +202,41 @@ def test_workspace_variant_bit_identical_and_deterministic(full_layer):
     assert torch.equal(y1, y3) and torch.equal(m1, m3)
 
 
+@pytest.mark.parametrize("T", [64, 300, 4096])
+def test_tensor_path_bit_identical_reruns(T, full_layer):
+    """Every sum on the tensor path has a fixed order (split-K partials
+    included), so repeated calls give the same bits; a race between the
+    pipelines' stages would show up here.  Back-to-back calls on one stream,
+    so each one's kernels overlap the previous one's tail."""
+    wl, host, dev = full_layer
+    x = make_tokens(WORKLOADS["prefill"], T=T, seed=21).to(DEV)
+    outs = [sfn.sparse_ffn_forward(x, dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"],
+                                   path="tensor") for _ in range(4)]
+    torch.cuda.synchronize()
+    for y, m in outs[1:]:
+        assert torch.equal(y, outs[0][0]) and torch.equal(m, outs[0][1])
+
+
+def test_concurrent_streams_match_serial(full_layer):
+    """Calls on two streams at once (each with its own stream-ordered
+    scratch) give the same bits as the same calls one after the other: the
+    library keeps no per-call state outside the caller's buffers."""
+    wl, host, dev = full_layer
+    args = (dev["A"], dev["B"], dev["Wg"], dev["Wu"], dev["Wd"])
+    xs = [make_tokens(WORKLOADS["prefill"], T=T, seed=30 + T).to(DEV) for T in (1, 64, 300)]
+    serial = [sfn.sparse_ffn_forward(x, *args) for x in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in xs]
+    conc = []
+    for x, s in zip(xs, streams):
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            conc.append(sfn.sparse_ffn_forward(x, *args))
+    torch.cuda.synchronize()
+    for (y1, m1), (y2, m2) in zip(serial, conc):
+        assert torch.equal(y1, y2) and torch.equal(m1, m2)
+
+
 def test_outputs_do_not_spill(full_layer):
     """Canary words around y and mask stay untouched; mask may be omitted."""
     wl, host, dev = full_layer
