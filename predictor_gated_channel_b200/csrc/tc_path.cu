@@ -30,7 +30,12 @@
 //               accumulator so the next tile's MMAs overlap this epilogue
 // With one token tile every weight byte is read once: the weight loads then
 // carry an evict-first L2 policy, and the producer issues the first stages'
-// weight loads before its dependency wait.
+// weight loads before its dependency wait.  There, G2 also runs inside G3
+// (k_tc_logits_gateup, below).  With few token tiles, G1 and G4 split K over
+// the SMs into ranges that differ by at most one block, and write float32
+// partials that a separate kernel sums in a fixed order.
+// The same engine runs the Dense-4x comparison's gate/up GEMM and the
+// backward's float32-output contractions (A and B K-major or MN-major).
 // Every mbarrier wait is bounded (async_util.cuh).
 #include <cudaTypedefs.h>
 
