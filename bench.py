@@ -184,13 +184,38 @@ KERNEL_SOURCES = {
 COMMON_SOURCES = ["sfn_internal.cuh", "async_util.cuh"]
 
 
+def _code_only(text):
+    """C/C++ source without comments and blank space, so that a digest
+    changes with the code and not with its comments."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_digest(kernel):
-    """Digest of the sources a stage's kernel is compiled from."""
+    """Digest of the code (comments left out) a stage's kernel is compiled
+    from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "predictor_gated_channel_b200", "csrc")
     for name in sorted(KERNEL_SOURCES.get(kernel, []) + COMMON_SOURCES):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:12]
 
 
