@@ -125,3 +125,18 @@ def test_bank_sharded_layer_allreduce_gloo():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert all(ok and mask_ok for _, ok, mask_ok in res)
+
+
+def test_traffic_digest_ignores_comments_only():
+    """The DRAM-traffic figures in profiles/ stay valid across comment edits
+    and lapse with any change to the code they were measured on (bench.py
+    then reports the traffic as null)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    code = 'int f(int a) { return a + 1; } /* tail */ const char *s = "// kept";\n'
+    commented = ("// header\nint f(int a) {  // adds one\n  return a + 1;\n}\n"
+                 "/* tail */ const char *s = \"// kept\";\n")
+    assert bench._code_only(code) == bench._code_only(commented)
+    assert bench._code_only(code) != bench._code_only(code.replace("+ 1", "+ 2"))
+    assert "// kept" in bench._code_only(commented)
