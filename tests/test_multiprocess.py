@@ -1,4 +1,5 @@
-"""Multi-rank host logic of bench.py on CPU (gloo, world size 2).
+"""Host logic of bench.py on CPU: the multi-rank parts (gloo, world size 2),
+the traffic digests and the roofline accounting.
 
 The path shards by tokens with no collective on the data path; the only
 cross-rank step is the max over ranks of the timed region (the slowest rank
@@ -140,3 +141,31 @@ def test_traffic_digest_ignores_comments_only():
     assert bench._code_only(code) == bench._code_only(commented)
     assert bench._code_only(code) != bench._code_only(code.replace("+ 1", "+ 2"))
     assert "// kept" in bench._code_only(commented)
+
+
+def test_roofline_accounting_matches_the_layer_sizes():
+    """bench.py's algorithmic work per step against the totals the layer's
+    sizes fix (d 4096, d_i 14336, r 448, bank 64, k 16, bf16): a decode step
+    reads A (3.67 MB), B (12.85 MB) and three 8 KB rows per kept channel
+    (3584 of them), 104.6 MB in all, and does 104.6 MFLOP of useful work per
+    token (368.8 with every channel kept)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from predictor_gated_channel_b200.inputs import WORKLOADS
+    wl = WORKLOADS["decode"]
+    w = bench.stage_work(wl, 1, wl.d_s)
+    rows = 3 * 3584 * 8192
+    assert rows == 88_080_384
+    assert w["ffn"]["bytes"] - rows < 64 * 1024          # x, the kept ids and sigmas
+    step = sum(w[s]["bytes"] for s in ("pred_h", "logits_topk", "ffn", "reduce"))
+    assert abs(step - 104.6e6) < 0.15e6
+    assert w["pred_h"]["bytes"] >= 448 * 4096 * 2 and w["logits_topk"]["bytes"] >= 14336 * 448 * 2
+    assert abs(bench.useful_flops_per_token(wl) - 104.6e6) < 0.1e6
+    dense = bench.useful_flops_per_token(wl.with_(k=64))
+    assert abs(dense - 368.8e6) < 0.1e6
+    # 64 tokens whose masks cover every channel read every row once
+    w64 = bench.stage_work(wl, 64, wl.d_i)
+    weights = 3 * 14336 * 4096 * 2
+    gu_down = w64["tc_gateup"]["bytes"] + w64["tc_down"]["bytes"]
+    assert weights <= gu_down < weights + 8e6
